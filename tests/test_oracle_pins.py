@@ -1,0 +1,309 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test ties one part of the oracle to something other than itself: values
+printed on the pages (tests/golden), closed forms, library routines (torch
+float64) and brute-force enumeration written independently in Python.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand(shape, seed):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape)
+
+
+# --------------------------------------------------------------- worked example
+def test_worked_example_weighted_sum(oracle_mod):
+    """1cademy worked question: G={0,2}, alpha=0.6/0.4, v0=[1,0], v2=[0,3] -> [0.6, 1.2]."""
+    g = _golden("worked_example_1cademy.json")
+    V = np.array(g["V"])
+    out = oracle_mod.weighted_sum(g["G"], g["alpha"], V)
+    assert np.allclose(out, g["expected_out"], rtol=0, atol=1e-15)
+    # v_1 is not in G: changing it must not change the output.
+    V2 = V.copy()
+    V2[1] = [1e6, -1e6]
+    assert np.array_equal(oracle_mod.weighted_sum(g["G"], g["alpha"], V2), out)
+
+
+def test_worked_example_from_logits(oracle_mod):
+    """Same example reached through the softmax: logits ln(1.5) and 0 give 0.6/0.4."""
+    g = _golden("worked_example_1cademy.json")
+    d = 2
+    q = np.array([[[math.sqrt(2.0) * math.log(1.5), 0.0]]])          # [S=1][H=1][d]
+    K = np.zeros((1, 1, 4, d))
+    K[0, 0, 0] = [1.0, 0.0]                                           # s_0 = ln 1.5
+    K[0, 0, 1] = [5.0, 5.0]                                           # not in G
+    K[0, 0, 2] = [0.0, 0.0]                                           # s_2 = 0
+    V = np.zeros((1, 1, 4, d))
+    V[0, 0, :3] = g["V"]
+    V[0, 0, 3] = [7.0, 7.0]
+    idx = np.array([[g["G"]]], dtype=np.int32)
+    out, lse = oracle_mod.gather(q, K, V, idx)
+    assert np.allclose(out[0, 0], g["expected_out"], rtol=0, atol=1e-14)
+    assert abs(lse[0, 0] - math.log(2.5)) < 1e-14
+
+
+# ---------------------------------------------------------- dense equivalence
+def _torch_dense(Q, K, V, causal, scale):
+    q, k, v = (torch.from_numpy(x) for x in (Q, K, V))
+    g = q.shape[1] // k.shape[1]
+    k = k.repeat_interleave(g, dim=1)
+    v = v.repeat_interleave(g, dim=1)
+    s = (q @ k.transpose(-1, -2)) * scale
+    if causal:
+        n = s.shape[-1]
+        s = s.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    return (torch.softmax(s, dim=-1) @ v).numpy()
+
+
+@pytest.mark.parametrize("causal", [0, 1])
+def test_full_G_is_dense_attention(oracle_mod, causal):
+    """A full G (no primitive) reproduces softmax(QK^T/sqrt(d))V (glossary formula)."""
+    B, H, Hkv, N, d = 2, 4, 2, 37, 8
+    Q, K, V = _rand((B, H, N, d), 1), _rand((B, Hkv, N, d), 2), _rand((B, Hkv, N, d), 3)
+    p = oracle_mod.Pattern(causal=causal)
+    O, lse = oracle_mod.prefill(p, Q, K, V)
+    Od = oracle_mod.dense(Q, K, V, causal=bool(causal))
+    Ot = _torch_dense(Q, K, V, causal, 1 / math.sqrt(d))
+    assert np.max(np.abs(O - Od)) < 1e-12
+    assert np.max(np.abs(O - Ot)) < 1e-12
+
+
+def test_gqa_equals_mha_on_repeated_kv(oracle_mod):
+    """GQA with contiguous head groups == MHA on repeat_interleave'd K/V."""
+    B, H, Hkv, N, d = 1, 6, 2, 40, 8
+    Q, K, V = _rand((B, H, N, d), 4), _rand((B, Hkv, N, d), 5), _rand((B, Hkv, N, d), 6)
+    p = oracle_mod.Pattern(causal=1, window=7, n_global=2, block_q=64, block_k=64)
+    O1, _ = oracle_mod.prefill(p, Q, K, V)
+    Kr, Vr = np.repeat(K, H // Hkv, axis=1), np.repeat(V, H // Hkv, axis=1)
+    O2, _ = oracle_mod.prefill(p, Q, Kr, Vr)
+    assert np.array_equal(O1, O2)
+
+
+# ---------------------------------------------------------------- G enumeration
+def _patterns(oracle_mod, N, H):
+    tab = np.stack([np.sort(np.random.default_rng(7 + h).choice(-(-N // 64), size=(-(-N // 64), 2),
+                                                                  replace=True), axis=-1)
+                    for h in range(H)]).astype(np.int32)
+    # make entries distinct per row
+    for h in range(H):
+        for r in range(tab.shape[1]):
+            if tab[h, r, 0] == tab[h, r, 1]:
+                tab[h, r, 1] = (tab[h, r, 0] + 1) % tab.shape[1]
+    P = oracle_mod.Pattern
+    return [
+        P(),
+        P(causal=1),
+        P(causal=1, window=5),
+        P(causal=0, window=6),
+        P(causal=0, window=7),
+        P(causal=1, window=9, n_global=3),
+        P(causal=0, window=4, n_global=2),
+        P(causal=0, block_local=16),
+        P(causal=1, block_local=32, window=3),
+        P(causal=0, n_random=2, random_block=64, random_table=tab),
+        P(causal=1, n_global=1, n_random=2, random_block=64, random_table=tab),
+        P(causal=0, window=10, n_global=5, n_random=2, random_block=64, random_table=tab),
+    ]
+
+
+@pytest.mark.parametrize("N", [1, 50, 130])
+def test_G_ranges_equal_bruteforce(oracle_mod, N):
+    """Range construction == C predicate == an independent Python predicate."""
+    H = 2
+    for p in _patterns(oracle_mod, N, H):
+        for h in range(H):
+            for i in range(N):
+                G = oracle_mod.build_G(p, N, h, i).tolist()
+                brute = [j for j in range(N) if oracle_mod.visible_py(p, N, h, i, j)]
+                assert G == brute, (p, h, i)
+                cpred = [j for j in range(N) if oracle_mod.visible(p, N, h, i, j)]
+                assert G == cpred
+
+
+def test_window_closed_form(oracle_mod):
+    """Mistral rule: |G_i| = min(i + 1, W) for the causal window [max(0, i-W+1), i]."""
+    N, W = 300, 64
+    p = oracle_mod.Pattern(causal=1, window=W)
+    for i in range(N):
+        assert len(oracle_mod.build_G(p, N, 0, i)) == min(i + 1, W)
+
+
+def test_tiny_static_pair_count(oracle_mod):
+    """causal and (window 64 or globals 0..3), N=256: 15,130 pairs per head (closed form)."""
+    N, W, g = 256, 64, 4
+    p = oracle_mod.Pattern(causal=1, window=W, n_global=g, block_q=64, block_k=64)
+    total = sum(len(oracle_mod.build_G(p, N, 0, i)) for i in range(N))
+    closed = sum(i + 1 for i in range(W)) + sum(W + sum(1 for j in range(g) if j < i - W + 1)
+                                                 for i in range(W, N))
+    assert total == closed == 15130
+
+
+def test_page_counts(oracle_mod):
+    c = _golden("counts.json")
+    # dense 5x5: no primitive, non-causal -> all 25 pairs
+    p = oracle_mod.Pattern()
+    assert sum(len(oracle_mod.build_G(p, 5, 0, i)) for i in range(5)) == c["dense_5x5"]["pairs"]
+    # explicit sparse grid: 10 pairs, a 60% reduction; rows through the explicit-set entry
+    sp = c["sparse_5x5"]
+    assert sum(len(s) for s in sp["G"]) == sp["pairs"]
+    assert 1 - sp["pairs"] / c["dense_5x5"]["pairs"] == pytest.approx(sp["reduction"])
+    # first token + itself + two preceding: causal window 3 or global 1
+    fp = c["first_plus_local"]
+    p = oracle_mod.Pattern(causal=1, window=3, n_global=1)
+    G = oracle_mod.build_G(p, fp["N"], 0, fp["i"])
+    assert len(G) == fp["pairs"] and G.tolist() == [0, fp["i"] - 2, fp["i"] - 1, fp["i"]]
+
+
+def test_explicit_sets_row_softmax(oracle_mod):
+    """Explicit sets (the 5x5 grid) -- each row is the softmax over exactly its set."""
+    c = _golden("counts.json")["sparse_5x5"]
+    d = 3
+    Q = _rand((5, d), 11)
+    K = _rand((5, d), 12)
+    V = _rand((5, d), 13)
+    for i, G in enumerate(c["G"]):
+        idx = np.array([[G]], dtype=np.int32)
+        out, _ = oracle_mod.gather(Q[i][None, None], K[None, None], V[None, None], idx)
+        s = np.array([Q[i] @ K[j] / math.sqrt(d) for j in G])
+        a = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
+        assert np.allclose(out[0, 0], sum(a[k] * V[j] for k, j in enumerate(G)), atol=1e-14)
+
+
+def test_exclusion(oracle_mod):
+    """1cademy: j outside G_i contributes nothing -- perturbing those K/V rows leaves out_i."""
+    B, H, Hkv, N, d = 1, 2, 2, 96, 8
+    Q, K, V = _rand((B, H, N, d), 21), _rand((B, Hkv, N, d), 22), _rand((B, Hkv, N, d), 23)
+    p = oracle_mod.Pattern(causal=1, window=8, n_global=2, block_q=64, block_k=64)
+    i = 70
+    rows = np.array([[0, h, i] for h in range(H)], np.int32)
+    O1, _ = oracle_mod.prefill(p, Q, K, V, rows=rows)
+    G = set(oracle_mod.build_G(p, N, 0, i).tolist())
+    K2, V2 = K.copy(), V.copy()
+    for j in range(N):
+        if j not in G:
+            K2[:, :, j] += 100.0
+            V2[:, :, j] -= 100.0
+    O2, _ = oracle_mod.prefill(p, Q, K2, V2, rows=rows)
+    assert np.array_equal(O1, O2)
+
+
+# ------------------------------------------------------------- block-skip rule
+def _bsfa_small(oracle_mod, seed=31):
+    B, H, Hkv, N, d = 1, 2, 1, 512, 16
+    Q, K, V = _rand((B, H, N, d), seed), _rand((B, Hkv, N, d), seed + 1), _rand((B, Hkv, N, d), seed + 2)
+    return B, H, Hkv, N, d, Q, K, V
+
+
+def test_tile_statistic_bruteforce(oracle_mod):
+    """Block statistic, pair count and fullness of a tile against numpy brute force."""
+    B, H, Hkv, N, d, Q, K, V = _bsfa_small(oracle_mod)
+    p = oracle_mod.Pattern(causal=1, window=150, block_q=128, block_k=64)
+    scale = 1 / math.sqrt(d)
+    for t in range(N // 128):
+        cnt, full, stat, mask = oracle_mod.tile_blocks(p, Q, K, 0, 1, t)
+        for kb in range(N // 64):
+            vals = [scale * Q[0, 1, i] @ K[0, 0, j]
+                    for i in range(t * 128, t * 128 + 128) for j in range(kb * 64, kb * 64 + 64)
+                    if oracle_mod.visible_py(p, N, 1, i, j)]
+            assert cnt[kb] == len(vals)
+            assert full[kb] == (len(vals) == 128 * 64)
+            if vals:
+                assert stat[kb] == pytest.approx(max(vals), abs=1e-12)
+                assert mask[kb] == 1
+            else:
+                assert mask[kb] == 0
+
+
+def test_bsfa_threshold_minus_inf_is_dense(oracle_mod):
+    """tau = -inf skips nothing: identical to exact causal attention."""
+    B, H, Hkv, N, d, Q, K, V = _bsfa_small(oracle_mod)
+    p = oracle_mod.Pattern(causal=1, block_q=128, block_k=64)
+    O0, l0 = oracle_mod.prefill(p, Q, K, V)
+    O1, l1, mask, stat, full = oracle_mod.prefill(p, Q, K, V, thresholds=np.full(H, -np.inf),
+                                                  want_blocks=True)
+    assert np.array_equal(O0, O1) and np.array_equal(l0, l1)
+    assert not (mask == 2).any()
+    assert np.max(np.abs(O0 - _torch_dense(Q, K, V, 1, 1 / math.sqrt(d)))) < 1e-12
+
+
+def test_bsfa_threshold_plus_inf_keeps_partial_blocks_only(oracle_mod):
+    """tau = +inf skips every full block; what is left is the diagonal 128x128 block."""
+    B, H, Hkv, N, d, Q, K, V = _bsfa_small(oracle_mod)
+    p = oracle_mod.Pattern(causal=1, block_q=128, block_k=64)
+    O1, _, mask, _, full = oracle_mod.prefill(p, Q, K, V, thresholds=np.full(H, np.inf),
+                                              want_blocks=True)
+    assert ((mask == 2) == full).all()
+    diag = oracle_mod.Pattern(causal=1, block_local=128, block_q=128, block_k=64)
+    O2, _ = oracle_mod.prefill(diag, Q, K, V)
+    assert np.max(np.abs(O1 - O2)) < 1e-12
+
+
+def test_bsfa_calibrated_skip_fraction(oracle_mod):
+    """Lower-median threshold on the same draw skips floor((n-1)/2) of n full blocks per head."""
+    B, H, Hkv, N, d, Q, K, V = _bsfa_small(oracle_mod)
+    p = oracle_mod.Pattern(causal=1, block_q=128, block_k=64)
+    full, stat, _ = oracle_mod.block_stats(p, Q, K)
+    tau = oracle_mod.calibrate_thresholds(full, stat)
+    _, _, mask, _, _ = oracle_mod.prefill(p, Q, K, V, thresholds=tau, want_blocks=True)
+    for h in range(H):
+        n = int(full[:, h].sum())
+        assert n == sum(2 * t for t in range(N // 128))   # blocks left of each diagonal
+        assert int((mask[:, h] == 2).sum()) == (n - 1) // 2
+
+
+def test_bsfa_skipped_keys_leave_G(oracle_mod):
+    """A skipped block's keys leave G_i of every row of the tile (the rows then equal an
+    explicit-set computation without them)."""
+    B, H, Hkv, N, d, Q, K, V = _bsfa_small(oracle_mod, seed=41)
+    p = oracle_mod.Pattern(causal=1, block_q=128, block_k=64)
+    full, stat, _ = oracle_mod.block_stats(p, Q, K)
+    tau = oracle_mod.calibrate_thresholds(full, stat)
+    O, _, mask, _, _ = oracle_mod.prefill(p, Q, K, V, thresholds=tau, want_blocks=True)
+    for h in range(H):
+        for i in (200, 383, 500):
+            t = i // 128
+            G = [j for j in range(i + 1) if mask[0, h, t, j // 64] != 2]
+            idx = np.array([[G]], dtype=np.int32)
+            og, _ = oracle_mod.gather(Q[0, h][i][None, None], K[0][None, :, : i + 1],
+                                      V[0][None, :, : i + 1], idx)
+            assert np.max(np.abs(og[0, 0] - O[0, h, i])) < 1e-13
+
+
+def test_gather_equals_prefill_row(oracle_mod):
+    """With idx = static G_i of the last row, the explicit-set entry equals that prefill row."""
+    B, H, Hkv, N, d = 1, 4, 2, 200, 8
+    Q, K, V = _rand((B, H, N, d), 51), _rand((B, Hkv, N, d), 52), _rand((B, Hkv, N, d), 53)
+    p = oracle_mod.Pattern(causal=1, window=20, n_global=3)
+    i = N - 1
+    O, _ = oracle_mod.prefill(p, Q, K, V)
+    G = oracle_mod.build_G(p, N, 0, i)
+    idx = np.broadcast_to(G, (1, H, len(G))).astype(np.int32).copy()
+    og, _ = oracle_mod.gather(Q[:, :, i], K, V, idx)
+    assert np.max(np.abs(og[0] - O[0, :, i])) < 1e-14
+
+
+def test_bf16_inputs_convert_exactly(oracle_mod):
+    """bf16 inputs are converted exactly: the same values as float64 give identical output."""
+    B, H, N, d = 1, 1, 64, 8
+    g = torch.Generator().manual_seed(3)
+    Qb = torch.randn(B, H, N, d, generator=g).bfloat16()
+    Kb = torch.randn(B, H, N, d, generator=g).bfloat16()
+    Vb = torch.randn(B, H, N, d, generator=g).bfloat16()
+    p = oracle_mod.Pattern(causal=1, window=9)
+    O1, _ = oracle_mod.prefill(p, Qb, Kb, Vb)
+    O2, _ = oracle_mod.prefill(p, Qb.double().numpy(), Kb.double().numpy(), Vb.double().numpy())
+    assert np.array_equal(O1, O2)
