@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch of synthetic input: for a
+prefill workload one sparse_attn_prefill_plan launch (pattern compile and, for
+the block-skip workload, the one-time threshold calibration happen before the
+timed region); for gather_decode one sparse_attn_gather launch.
+
+Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
+and torch.cuda.synchronize() on both sides.  L2 is flushed (256 MiB write)
+before every step, outside the timed kernel window; each step's kernel is
+timed with CUDA events recorded on the stream it is launched on.  Multi-GPU
+(torchrun): every rank runs an independent replica (the path has no exchange
+step), the time is the max over ranks and `value` aggregates all ranks.
+
+The printed JSON line carries the headline metric, an end-to-end number
+through the same C-ABI call with host (pinned) buffers and the host<->device
+copies inside the timed region, the roofline of the dominant kernel against
+the measured peaks, SM clocks sampled during the timed region and the CPU
+baseline (the fp64 oracle on a bounded sample, rank 0, N=1 only).
+
+--impl reference times the fp64 CPU oracle as it stands on the host cores, on
+the same workload and metric (bounded samples per step), and prints the same
+JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers --
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "block_sparse_attention_29_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, sha):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    has not changed since it was captured."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t[kernel][workload]
+        if e.get("source_sha") == sha:
+            return e["dram_bytes_per_launch"]
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.samples, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for s in self.samples for k in range(4)
+                          if s[3 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- workloads --
+def prefill_accounting(w, info, kept_desc=None, skipped_pairs=0):
+    """FLOPs of one prefill launch: computed-block (descriptor granularity),
+    exact-pair and dense-equivalent."""
+    bq, bk, d = w.block_q, w.block_k, w.d
+    blocks = info["blocks_desc"]
+    kept = blocks if kept_desc is None else kept_desc
+    computed = 2 * bq * bk * d * (blocks + kept)
+    pairs = info["pairs"]
+    exact = 2 * d * pairs + 2 * d * (pairs - skipped_pairs)
+    p_dense = w.N * (w.N + 1) // 2 if w.causal else w.N * w.N
+    dense = 4 * w.B * w.H * d * p_dense
+    return computed, exact, dense
+
+
+def setup_prefill(w, device, torch, sa, workloads):
+    Q, K, V, tab = workloads.prefill_inputs(w, device=device)
+    pat = sa.Pattern(**w.pattern_fields(), random_table=tab)
+    plan = sa.Plan(pat, w.B, w.H, w.H_kv, w.N, w.d)
+    thresholds = None
+    extra = {"plan_compile_ms": round(plan.info["compile_ms"], 2)}
+    kept_desc, skipped_pairs = None, 0
+    if w.bsfa:
+        Qc, Kc, _, _ = workloads.calibration_inputs(w, device=device)
+        thresholds = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
+        del Qc, Kc
+        mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=device)
+        plan.prefill(Q, K, V, thresholds=thresholds, block_mask=mask)
+        sa.check_device_error()
+        skipped = int((mask == 2).sum())
+        kept_desc = plan.info["blocks_desc"] - skipped
+        skipped_pairs = skipped * w.block_q * w.block_k
+        extra["blocks_skipped"] = skipped
+        extra["skip_fraction_of_full"] = round(skipped / max(1, plan.info["blocks_full"]), 4)
+        extra["v_loads_issued_fraction"] = round(kept_desc / plan.info["blocks_desc"], 4)
+        del mask
+    computed, exact, dense = prefill_accounting(w, plan.info, kept_desc, skipped_pairs)
+    extra.update({"blocks_listed": plan.info["blocks_desc"], "pairs": plan.info["pairs"]})
+    O = torch.empty_like(Q)
+
+    def step(stream=None):
+        plan.prefill(Q, K, V, O=O, thresholds=thresholds, stream=stream)
+
+    def e2e_step(host, dev_bufs, stream):
+        Qd, Kd, Vd, Od = dev_bufs
+        Qd.copy_(host[0], non_blocking=True)
+        Kd.copy_(host[1], non_blocking=True)
+        Vd.copy_(host[2], non_blocking=True)
+        plan.prefill(Qd, Kd, Vd, O=Od, thresholds=thresholds, stream=stream)
+        host[3].copy_(Od, non_blocking=True)
+
+    host = [Q.cpu().pin_memory(), K.cpu().pin_memory(), V.cpu().pin_memory(),
+            torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)]
+    dev_bufs = [torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(O)]
+    h2d = sum(t.numel() * t.element_size() for t in host[:3])
+    d2h = host[3].numel() * host[3].element_size()
+    algo_bytes = sum(t.numel() * t.element_size() for t in (Q, K, V, O))
+    return dict(step=step, e2e_step=lambda s: e2e_step(host, dev_bufs, s), h2d=h2d, d2h=d2h,
+                flops=computed, exact_flops=exact, dense_flops=dense, algo_bytes=algo_bytes,
+                extra=extra, kernel="prefill_kernel", kernel_files=["prefill_sm100.cu"],
+                metric="effective TFLOP/s (computed blocks)", unit="TFLOP/s", bound="tensor",
+                tensors=(Q, K, V, O), plan=plan, tab=tab, thresholds=thresholds)
+
+
+def setup_gather(w, device, torch, sa, workloads):
+    Q, K, V, idx = workloads.gather_inputs(w, device=device)
+    O = torch.empty_like(Q)
+    n_sets = w.S * w.H
+    rows = n_sets * w.n_idx
+    algo_bytes = rows * 2 * w.d * 2 + idx.numel() * 4 + Q.numel() * 2 + O.numel() * 2
+    flops = 4 * rows * w.d
+
+    def step(stream=None):
+        sa.sparse_attn_gather(Q, K, V, idx, O=O, stream=stream)
+
+    # end to end: the query and index sets come from the host each step, the
+    # KV cache stays resident (it is the cache being decoded against)
+    host = [Q.cpu().pin_memory(), idx.cpu().pin_memory(),
+            torch.empty(O.shape, dtype=O.dtype, pin_memory=True)]
+    Qd, idxd, Od = torch.empty_like(Q), torch.empty_like(idx), torch.empty_like(O)
+
+    def e2e_step(stream):
+        Qd.copy_(host[0], non_blocking=True)
+        idxd.copy_(host[1], non_blocking=True)
+        sa.sparse_attn_gather(Qd, K, V, idxd, O=Od, stream=stream)
+        host[2].copy_(Od, non_blocking=True)
+
+    h2d = host[0].numel() * 2 + host[1].numel() * 4
+    d2h = host[2].numel() * 2
+    return dict(step=step, e2e_step=e2e_step, h2d=h2d, d2h=d2h, flops=flops, exact_flops=flops,
+                dense_flops=4 * n_sets * w.L * w.d, algo_bytes=algo_bytes,
+                extra={"rows_gathered": rows}, kernel="gather_kernel",
+                kernel_files=["gather_sm100.cu"], metric="gather GB/s", unit="GB/s", bound="hbm",
+                tensors=(Q, K, V, idx, O), idx=idx)
+
+
+# ------------------------------------------------------------- CPU baseline --
+def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
+    """Times the fp64 oracle as it stands on the host cores over a bounded sample
+    of the workload; returns (value in the workload's unit, cores, description)."""
+    import numpy as np
+    import torch
+    import oracle
+    from block_sparse_attention_29_b200 import workloads
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    g = np.random.default_rng(1234 + sample_seed)
+    if isinstance(w, workloads.GatherWorkload):
+        # gather: sampled (sequence, head) sets, only their referenced rows on the host
+        if device_tensors is None:
+            raise RuntimeError("gather baseline needs the device tensors")
+        Q, K, V, idx = device_tensors
+        group = w.H // w.H_kv
+        done_rows, t_total = 0, 0.0
+        n = 8
+        while t_total < seconds:
+            pairs = [(int(g.integers(w.S)), int(g.integers(w.H))) for _ in range(n)]
+            Qs = torch.stack([Q[s, h] for s, h in pairs])[None]
+            ixs = [idx[s, h if w.H_idx == w.H else h // group].long() for s, h in pairs]
+            Ks = torch.stack([K[s, h // group, ix] for (s, h), ix in zip(pairs, ixs)])[None]
+            Vs = torch.stack([V[s, h // group, ix] for (s, h), ix in zip(pairs, ixs)])[None]
+            # one "sequence" whose K/V heads are the sampled sets, one query head per set
+            local = np.broadcast_to(np.arange(w.n_idx, dtype=np.int32), (1, n, w.n_idx)).copy()
+            Qh, Kh, Vh = Qs.cpu(), Ks.cpu(), Vs.cpu()
+            t0 = time.perf_counter()
+            oracle.gather(Qh, Kh, Vh, local, nthreads=cores)
+            t_total += time.perf_counter() - t0
+            done_rows += n * w.n_idx
+            n = min(4096, n * 2)
+        gbs = done_rows * (2 * w.d * 2 + 4) / t_total / 1e9
+        return gbs, cores, f"{done_rows // w.n_idx} (sequence, head) sets, {done_rows} rows"
+    # prefill: whole 128-row tiles, so computed-block FLOPs are exact for the sample
+    Q, K, V, tab = (device_tensors if device_tensors is not None
+                    else workloads.prefill_inputs(w, device="cpu"))
+    if isinstance(Q, torch.Tensor):
+        Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
+    opat = oracle.Pattern(**w.pattern_fields(), random_table=tab)
+    thresholds = None
+    if w.bsfa:
+        thresholds = np.zeros(w.H)   # the rule's statistic pass is what is timed
+    from block_sparse_attention_29_b200 import compile_pattern, Pattern
+    row_ptr, kb, full, cnt, H_pat, T = compile_pattern(Pattern(**w.pattern_fields(),
+                                                               random_table=tab), w.H, w.N)
+    flops_done, t_total, tiles_done, n = 0, 0.0, 0, 1
+    while t_total < seconds:
+        tiles = [(int(g.integers(w.B)), int(g.integers(w.H)), int(g.integers(T))) for _ in range(n)]
+        rows = np.array([(b, h, i) for b, h, t in tiles
+                         for i in range(t * 128, min(w.N, t * 128 + 128))], np.int32)
+        t0 = time.perf_counter()
+        oracle.prefill(opat, Qh, Kh, Vh, thresholds=thresholds, rows=rows, nthreads=cores)
+        t_total += time.perf_counter() - t0
+        for b, h, t in tiles:
+            hp = h if H_pat > 1 else 0
+            nb = int(row_ptr[hp * T + t + 1] - row_ptr[hp * T + t])
+            flops_done += 4 * 128 * 64 * w.d * nb
+        tiles_done += n
+        n = min(64, n * 2)
+    return flops_done / t_total / 1e12, cores, f"{tiles_done} whole 128-row query tiles"
+
+
+# --------------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mistral_swa")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from block_sparse_attention_29_b200 import workloads
+    w = workloads.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        run_reference(args, w, world)
+        return
+
+    import torch
+    import block_sparse_attention_29_b200 as sa
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
+
+    setup = setup_gather if isinstance(w, workloads.GatherWorkload) else setup_prefill
+    S = setup(w, device, torch, sa, workloads)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        S["step"](stream)
+    sa.check_device_error()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            S["step"](stream)
+            ends[k].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    sa.check_device_error()
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(per_step)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    # end to end: the same call with host buffers, copies inside the timed region
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        S["e2e_step"](stream)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        S["e2e_step"](stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+    if dist:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item()) / args.steps
+    sa.check_device_error()
+
+    peaks, peak_src = load_peaks()
+    per_launch_s = ms_per_step / 1e3
+    if S["unit"] == "TFLOP/s":
+        value = world * S["flops"] / per_launch_s / 1e12
+        e2e_value = world * S["flops"] / (e2e_ms / 1e3) / 1e12
+        achieved = S["flops"] / per_launch_s / 1e12
+        peak = peaks["bf16_tflops"]
+        roof_unit = "TFLOP/s"
+    else:
+        value = world * S["algo_bytes"] / per_launch_s / 1e9
+        e2e_value = world * S["algo_bytes"] / (e2e_ms / 1e3) / 1e9
+        achieved = value / world
+        peak = peaks["hbm_gbs"]
+        roof_unit = "GB/s"
+    sha = kernel_source_sha(S["kernel_files"])
+    traffic = recorded_traffic(S["kernel"], w.name, sha)
+
+    out = {
+        "metric": S["metric"], "value": round(value, 3), "unit": S["unit"], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, device-generated; see block_sparse_attention_29_b200/workloads.py)",
+        "config": config_of(w, world),
+        "e2e": {"value": round(e2e_value, 3), "unit": S["unit"],
+                "h2d_bytes_per_step": S["h2d"], "d2h_bytes_per_step": S["d2h"],
+                "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": S["bound"], "achieved": round(achieved, 3), "peak": peak,
+                     "unit": roof_unit, "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if roof_unit == 'TFLOP/s' else 'hbm_gbs'})",
+                     "traffic": traffic, "kernel": S["kernel"], "kernel_source_sha": sha},
+        "clocks": clk.summary(),
+        "per_step_ms": {"min": round(min(per_step), 5), "median": round(statistics.median(per_step), 5),
+                        "max": round(max(per_step), 5)},
+    }
+    if S["unit"] == "TFLOP/s":
+        out["secondary"] = {
+            "dense_equiv_tflops": round(world * S["dense_flops"] / per_launch_s / 1e12, 3),
+            "exact_pair_tflops": round(world * S["exact_flops"] / per_launch_s / 1e12, 3),
+            "pct_bf16_peak_burst": round(100 * achieved / peaks["bf16_tflops"], 2),
+            "pct_bf16_peak_sustained": round(100 * achieved / peaks.get("bf16_tflops_sustained", 1400.0), 2),
+            "computed_block_flops": S["flops"], **S["extra"]}
+    else:
+        out["secondary"] = {"pct_hbm_peak": round(100 * achieved / peaks["hbm_gbs"], 2),
+                            "algorithmic_bytes": S["algo_bytes"], **S["extra"]}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if isinstance(w, workloads.GatherWorkload):
+            Q, K, V, idx, _ = S["tensors"]
+            dt = (Q, K, V, idx)
+        else:
+            Q, K, V, _ = S["tensors"]
+            dt = (Q, K, V, S["tab"])
+        val, cores, sample = cpu_oracle_rate(w, args.cpu_seconds, device_tensors=dt)
+        out["cpu_baseline"] = {"value": round(val, 6), "unit": S["unit"], "cores": cores,
+                               "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+def config_of(w, world):
+    from block_sparse_attention_29_b200 import workloads
+    if isinstance(w, workloads.GatherWorkload):
+        return {"workload": w.name, "sequences": w.S, "H": w.H, "H_kv": w.H_kv, "d": w.d,
+                "cache_len": w.L, "n_idx": w.n_idx, "H_idx": w.H_idx,
+                "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}
+    pat = {k: v for k, v in w.pattern_fields().items() if v}
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
+            "pattern": pat, "block_skip_rule": bool(w.bsfa),
+            "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}
+
+
+def run_reference(args, w, world):
+    """The fp64 oracle as it stands, on this host's cores (rank 0 only)."""
+    import oracle
+    oracle.build()
+    from block_sparse_attention_29_b200 import workloads
+    dt = None
+    if isinstance(w, workloads.GatherWorkload):
+        # a cache of the full size does not fit the host budget of this arm: the
+        # sampled sets' rows are drawn with the same recipe at reduced length
+        import dataclasses
+        import torch
+        ws = dataclasses.replace(w, S=4, L=max(w.n_idx + w.n_recent + 1, 8192))
+        Q, K, V, idx = workloads.gather_inputs(ws, device="cpu")
+        dt = (Q, K, V, idx)
+        w = ws
+    else:
+        dt = workloads.prefill_inputs(w, device="cpu")
+    budget = 60.0
+    per_step = max(1.0, budget / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_oracle_rate(w, per_step / 4, device_tensors=dt)
+    vals, cores, sample = [], None, None
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        v, cores, sample = cpu_oracle_rate(w, per_step, sample_seed=k + 1, device_tensors=dt)
+        vals.append(v)
+    elapsed = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    unit = "GB/s" if isinstance(w, workloads.GatherWorkload) else "TFLOP/s"
+    metric = "gather GB/s" if unit == "GB/s" else "effective TFLOP/s (computed blocks)"
+    out = {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(1e3 * elapsed / args.steps, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": config_of(w, world),
+           "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores,
+                            "kind": "oracle", "sample": f"per step: {sample}"},
+           "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

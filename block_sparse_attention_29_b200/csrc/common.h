@@ -1,0 +1,99 @@
+// common.h -- internal declarations shared by the library's translation units:
+// error reporting (host message + device error word), kernel parameter blocks
+// and launcher prototypes.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <vector>
+
+#include "../../include/sparse_attn.h"
+
+namespace sa {
+
+// ---------------------------------------------------------------- errors --
+// Host: set the thread-local message returned by sparse_attn_last_error().
+int set_error(int code, const char* fmt, ...);
+int cuda_error(cudaError_t e, const char* what);
+
+// Device error word (one per device, owned by the API translation unit and
+// passed to every kernel): 0 = none; otherwise (where << 8) | code of the
+// first error recorded since the last sparse_attn_check_device_error().
+int* device_error_word();   // host: address for the current device, or null
+
+__device__ __forceinline__ void record_device_error(int* err, int code, int where) {
+  atomicCAS(err, 0, (where << 8) | code);
+}
+
+// ---------------------------------------------------------------- prefill --
+constexpr int kTileQ = 128;   // query rows per tile (UMMA M)
+constexpr int kTileK = 64;    // keys per block (UMMA N of Q K^T)
+
+// Block-list entry: (kb << 1) | partial.
+__host__ __device__ inline int32_t entry_pack(int32_t kb, bool partial) {
+  return (kb << 1) | (partial ? 1 : 0);
+}
+
+struct PrefillParams {
+  CUtensorMap tm_q;   // 3-D {d, N, B*H}    box {64, 128, 1}, 128-B swizzle
+  CUtensorMap tm_k;   // 3-D {d, N, B*H_kv} box {64, 64, 1},  128-B swizzle
+  CUtensorMap tm_v;   // same as tm_k over V
+  uint16_t* O;        // [B][H][N][d] bf16
+  float* lse;         // [B][H][N] or null
+  uint8_t* mask_out;  // [B][H][T][n_kb] or null
+  float* stat_out;    // [B][H][T][n_kb] or null
+  const int32_t* row_ptr;   // [H_pat*T + 1]
+  const int32_t* entries;   // block lists
+  const int32_t* units;     // work order: unit = (b*H + h)*T + t
+  const int32_t* rtab;      // random table [H][n_rb][n_random] or null
+  const float* thresholds;  // [H] or null
+  int n_units;
+  int B, H, Hkv, N, T, n_kb, head_pat;   // head_pat: 1 when lists are per head
+  int causal, window, n_global, block_local, random_block, n_random;
+  int gate;        // 1: statistics + decision per block (rule or stats pass)
+  int stats_only;  // 1: no PV, no output (statistics pass)
+  int want_stats;  // 1: block statistics needed (stat_out or gate)
+  float scale;       // logit scale
+  float scale_log2;  // scale * log2(e)
+  int* err;          // device error word
+};
+
+int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
+
+// ----------------------------------------------------------------- gather --
+struct GatherParams {
+  const uint16_t* Q;   // [S][H][d]
+  const uint16_t* K;   // [S][H_kv][L][d]
+  const uint16_t* V;
+  const int32_t* idx;  // [S][H_idx][n_idx]
+  const int32_t* idx_len;  // [S][H_idx] or null
+  uint16_t* O;         // [S][H][d]
+  float* lse;          // [S][H] or null
+  int S, H, Hkv, H_idx, L, n_idx;
+  float scale_log2;
+  int* err;            // device error word
+};
+
+int launch_gather(const GatherParams& p, int d, cudaStream_t stream);
+
+// ------------------------------------------------------------ calibration --
+// Per-head rank selection over the statistics of full blocks (plan lists).
+int launch_calibrate(const float* stat, const int32_t* row_ptr, const int32_t* entries,
+                     int head_pat, int B, int H, int T, int n_kb, double q, float* out,
+                     cudaStream_t stream);
+
+// ------------------------------------------------------ pattern compiler --
+struct CompiledPattern {
+  int H_pat = 0, T = 0, n_kb = 0;
+  std::vector<int32_t> row_ptr;   // [H_pat*T + 1]
+  std::vector<int32_t> kb;        // listed key blocks, ascending per list
+  std::vector<uint8_t> full;      // every pair of the block is in G
+  std::vector<int64_t> cnt;       // visible pairs per listed block
+};
+// Returns SA_OK or an error code (message set).
+int compile_pattern(const sa_pattern_t* pat, int H, int N, int tile_q, int tile_k,
+                    CompiledPattern* out);
+// Validates the descriptor fields that do not depend on the kernel.
+int validate_pattern(const sa_pattern_t* pat, int H, int N);
+
+}  // namespace sa

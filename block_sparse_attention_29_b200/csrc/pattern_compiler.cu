@@ -1,0 +1,154 @@
+// pattern_compiler.cu -- host compiler from a static pattern descriptor to
+// per-(head, query tile) lists of key blocks.
+//
+// A row's visible keys are the union, by logical OR ("SAS: Sparse Attention
+// Synthesizer", Step 5, component 2), of the primitives of the glossary's
+// "Sparse Attention Patterns" table (sliding window with the Mistral rule,
+// global tokens, blockwise, BigBird random blocks), capped by the causal
+// constraint G_i in {0..i} ("Sparse Attention Weights Assumption").  Each
+// primitive contributes one index range per row (random blocks n_random
+// ranges), so a tile's per-block pair counts come from range arithmetic: a
+// difference array adds tile_k to every block a range covers completely and
+// the two edge blocks get their partial lengths.  A block is listed when it
+// holds at least one visible pair and is "full" when it holds tile_q*tile_k
+// (every pair of the tile, which also rules out ragged tiles and blocks).
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "common.h"
+
+namespace sa {
+
+namespace {
+struct Range {
+  int64_t lo, hi;  // [lo, hi)
+};
+
+bool random_on(const sa_pattern_t* p) {
+  return p->n_random > 0 && p->random_table != nullptr && p->random_block > 0;
+}
+
+// Visible key ranges of row i (unsorted, may overlap), before the causal cap.
+int row_ranges(const sa_pattern_t* p, int N, int h, int i, Range* r) {
+  int n = 0;
+  bool any = false;
+  if (p->window > 0) {
+    any = true;
+    if (p->causal) r[n++] = {int64_t(i) - p->window + 1, int64_t(i) + 1};
+    else r[n++] = {int64_t(i) - p->window / 2, int64_t(i) + p->window / 2 + 1};
+  }
+  if (p->n_global > 0) {
+    any = true;
+    r[n++] = {0, i < p->n_global ? int64_t(N) : int64_t(p->n_global)};
+  }
+  if (p->block_local > 0) {
+    any = true;
+    int64_t lo = int64_t(i / p->block_local) * p->block_local;
+    r[n++] = {lo, lo + p->block_local};
+  }
+  if (random_on(p)) {
+    any = true;
+    int nrb = (N + p->random_block - 1) / p->random_block;
+    const int32_t* row =
+        p->random_table + (int64_t(h) * nrb + i / p->random_block) * p->n_random;
+    for (int k = 0; k < p->n_random; ++k) {
+      int64_t lo = int64_t(row[k]) * p->random_block;
+      r[n++] = {lo, lo + p->random_block};
+    }
+  }
+  if (!any) r[n++] = {0, N};
+  return n;
+}
+}  // namespace
+
+int validate_pattern(const sa_pattern_t* p, int H, int N) {
+  if (!p) return set_error(SA_ERR_INVALID_ARG, "pattern descriptor is NULL");
+  if (H <= 0 || N <= 0) return set_error(SA_ERR_INVALID_ARG, "H and N must be positive");
+  if (p->window < 0 || p->n_global < 0 || p->block_local < 0 || p->n_random < 0)
+    return set_error(SA_ERR_INVALID_ARG, "negative pattern field");
+  if (p->block_q <= 0 || p->block_k <= 0)
+    return set_error(SA_ERR_INVALID_ARG, "block_q and block_k must be positive");
+  if (p->n_random > 0 && p->random_table != nullptr) {
+    if (p->random_block <= 0)
+      return set_error(SA_ERR_INVALID_ARG, "random_block must be positive");
+    int nrb = (N + p->random_block - 1) / p->random_block;
+    int64_t n = int64_t(H) * nrb * p->n_random;
+    for (int64_t k = 0; k < n; ++k) {
+      int32_t v = p->random_table[k];
+      if (v < 0 || v >= nrb)
+        return set_error(SA_ERR_INVALID_ARG, "random_table[%lld] = %d outside [0, %d)",
+                         (long long)k, v, nrb);
+    }
+  }
+  return SA_OK;
+}
+
+int compile_pattern(const sa_pattern_t* p, int H, int N, int tile_q, int tile_k,
+                    CompiledPattern* out) {
+  int rc = validate_pattern(p, H, N);
+  if (rc) return rc;
+  if (tile_q <= 0 || tile_k <= 0) return set_error(SA_ERR_INVALID_ARG, "bad tile size");
+  const int H_pat = random_on(p) ? H : 1;
+  const int T = (N + tile_q - 1) / tile_q;
+  const int n_kb = (N + tile_k - 1) / tile_k;
+  out->H_pat = H_pat;
+  out->T = T;
+  out->n_kb = n_kb;
+  out->row_ptr.assign(size_t(H_pat) * T + 1, 0);
+  out->kb.clear();
+  out->full.clear();
+  out->cnt.clear();
+
+  std::vector<Range> ranges(4 + (random_on(p) ? p->n_random : 0));
+  std::vector<int64_t> direct(n_kb), diff(n_kb + 1);
+  const int64_t full_pairs = int64_t(tile_q) * tile_k;
+  for (int hp = 0; hp < H_pat; ++hp) {
+    for (int t = 0; t < T; ++t) {
+      std::fill(direct.begin(), direct.end(), 0);
+      std::fill(diff.begin(), diff.end(), 0);
+      const int i0 = t * tile_q, i1 = std::min(N, i0 + tile_q);
+      for (int i = i0; i < i1; ++i) {
+        int nr = row_ranges(p, N, hp, i, ranges.data());
+        std::sort(ranges.begin(), ranges.begin() + nr,
+                  [](const Range& a, const Range& b) { return a.lo < b.lo; });
+        const int64_t cap = p->causal ? std::min<int64_t>(int64_t(i) + 1, N) : int64_t(N);
+        int64_t next = 0;  // keys below `next` are already counted for this row
+        for (int k = 0; k < nr; ++k) {
+          int64_t lo = std::max<int64_t>(std::max<int64_t>(ranges[k].lo, next), 0);
+          int64_t hi = std::min<int64_t>(ranges[k].hi, cap);
+          if (hi > lo) {
+            int64_t b0 = lo / tile_k, b1 = (hi - 1) / tile_k;
+            if (b0 == b1) {
+              direct[b0] += hi - lo;
+            } else {
+              direct[b0] += (b0 + 1) * tile_k - lo;
+              direct[b1] += hi - b1 * tile_k;
+              diff[b0 + 1] += tile_k;
+              diff[b1] -= tile_k;
+            }
+          }
+          next = std::max(next, hi);
+        }
+      }
+      int64_t run = 0;
+      for (int b = 0; b < n_kb; ++b) {
+        run += diff[b];
+        int64_t c = direct[b] + run;
+        if (c > 0) {
+          out->kb.push_back(b);
+          out->full.push_back(c == full_pairs ? 1 : 0);
+          out->cnt.push_back(c);
+        }
+      }
+      size_t row = size_t(hp) * T + t;
+      if (out->kb.size() > size_t(INT32_MAX))
+        return set_error(SA_ERR_NO_MEMORY, "block list longer than 2^31 entries");
+      out->row_ptr[row + 1] = int32_t(out->kb.size());
+    }
+  }
+  return SA_OK;
+}
+
+}  // namespace sa

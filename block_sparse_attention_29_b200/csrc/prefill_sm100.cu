@@ -1,0 +1,572 @@
+// prefill_sm100.cu -- block-sparse attention prefill for B200 (sm_100a).
+//
+// Computes out_i = sum_{j in G_i} softmax_G(s_ij) v_j ("Sparse Attention
+// Weights Assumption", sparse attention output formula) for every query row,
+// where G_i is given by per-(head, 128-row tile) lists of 64-key blocks built
+// by the host pattern compiler, optionally pruned by the Block-Sparse-
+// FlashAttention rule ("Block Sparse Flash Attention", paper summary and
+// improvements): the exact QK^T tile of a block is computed first, its
+// maximum scaled logit is compared with the head's calibrated threshold, and
+// below it the block's V tile is never loaded and its PV product never issued.
+//
+// One CTA = 6 warps, persistent, two CTAs per SM (each owns 256 TMEM columns):
+//   warp 0      TMA producer: Q tile once per work unit, K blocks in a ring.
+//   warp 1      TMEM owner and single-thread tcgen05 issuer: S = Q K^T into one
+//               of two TMEM S buffers, O += P V with P read from TMEM; it also
+//               issues the V tile loads, after the gate has kept the block.
+//   warps 2..5  softmax warpgroup, one query row per thread (TMEM lane):
+//               mask of partial blocks, row max, tile max and gate, online
+//               softmax statistics (m, l) in fp32, P (bf16) written back over
+//               S in TMEM, lazy rescale of O, epilogue O / l.
+// Work units (b, h, tile) are taken in a longest-first order computed on the
+// host; CTA c takes units c, c + grid, c + 2*grid, ...
+//
+// TMEM columns: S buffer 0 at [0, 64), S buffer 1 at [64, 128), O at
+// [128, 128 + d).  P of a block overwrites the first 32 columns of its S
+// buffer (bf16 pairs).
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "common.h"
+#include "ptx.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 256;
+constexpr int kTmemO = 128;
+constexpr uint32_t kSoftmaxBar = 1;    // named barrier of the softmax warpgroup
+constexpr float kRescaleLog2 = 8.0f;   // lazy rescale: keep a stale max up to 2^8
+
+// where-codes recorded with SA_ERR_TIMEOUT
+enum { W_PROD_Q = 1, W_PROD_K, W_MMA_Q, W_MMA_SFREE, W_MMA_K, W_MMA_VEMPTY, W_MMA_DEC,
+       W_MMA_P, W_MMA_VFULL, W_SM_S, W_SM_O, W_SM_EPI };
+
+template <int D>
+struct Cfg {
+  static constexpr int KS = D == 128 ? 2 : 3;   // K ring depth
+  static constexpr int VS = D == 128 ? 2 : 3;   // V ring depth
+  static constexpr int CH = D / 64;             // 64-column (128-byte) chunks per row
+  static constexpr int Q_BYTES = kTileQ * D * 2;
+  static constexpr int KV_BYTES = kTileK * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + KS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VS * KV_BYTES;
+  static constexpr int BAR_BYTES = 1024;
+  // At least 80 KB so that no third CTA fits on an SM: two CTAs use all 512
+  // TMEM columns, a third would block in tcgen05.alloc.
+  static constexpr int SMEM_USED = OFF_BAR + BAR_BYTES;
+  static constexpr int SMEM = (SMEM_USED > 80 * 1024 ? SMEM_USED : 80 * 1024) + 1024;
+};
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[3], k_empty[3];
+  uint64_t v_full[3], v_empty[3];
+  uint64_t s_full[2], s_free[2], p_ready[2], dec[2];
+  uint64_t o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  uint32_t flags[2];   // per S buffer: 1 = block kept, 0 = skipped
+  float red[2][4];     // per S buffer: warp maxima for the tile maximum
+};
+static_assert(sizeof(Bars) <= 1024, "barrier block too large");
+
+struct Unit {
+  int b, h, hkv, t, beg, n;
+};
+
+__device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
+  Unit u;
+  const int id = __ldg(p.units + ui);
+  u.t = id % p.T;
+  const int bh = id / p.T;
+  u.h = bh % p.H;
+  u.b = bh / p.H;
+  u.hkv = u.h / (p.H / p.Hkv);
+  const int row = (p.head_pat ? u.h : 0) * p.T + u.t;
+  u.beg = __ldg(p.row_ptr + row);
+  u.n = __ldg(p.row_ptr + row + 1) - u.beg;
+  return u;
+}
+
+// ------------------------------------------------------------ producer --
+template <int D>
+__device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars) {
+  using C = Cfg<D>;
+  volatile int* abort_flag = &bars->abort;
+  const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t sK = smem_u32(smem + C::OFF_K);
+  uint32_t qc = 0, kc = 0;
+  for (int ui = blockIdx.x; ui < p.n_units; ui += gridDim.x) {
+    const Unit u = get_unit(p, ui);
+    if (u.n == 0) continue;
+    if (!wait_bounded(smem_u32(&bars->q_empty), (qc & 1) ^ 1, abort_flag, p.err, W_PROD_Q))
+      goto drain;
+    mbar_expect_tx(smem_u32(&bars->q_full), C::Q_BYTES);
+    for (int c = 0; c < C::CH; ++c)
+      tma_load_3d(sQ + c * (kTileQ * 128), &p.tm_q, smem_u32(&bars->q_full), c * 64,
+                  u.t * kTileQ, u.b * p.H + u.h);
+    ++qc;
+    for (int k = 0; k < u.n; ++k) {
+      const int kb = __ldg(p.entries + u.beg + k) >> 1;
+      const int st = kc % C::KS;
+      if (!wait_bounded(smem_u32(&bars->k_empty[st]), ((kc / C::KS) & 1) ^ 1, abort_flag, p.err,
+                        W_PROD_K))
+        goto drain;
+      const uint32_t dst = sK + st * C::KV_BYTES;
+      mbar_expect_tx(smem_u32(&bars->k_full[st]), C::KV_BYTES);
+      for (int c = 0; c < C::CH; ++c)
+        tma_load_3d(dst + c * (kTileK * 128), &p.tm_k, smem_u32(&bars->k_full[st]), c * 64,
+                    kb * kTileK, u.b * p.Hkv + u.hkv);
+      ++kc;
+    }
+  }
+  return;
+drain:
+  // Let the loads already issued land before the CTA's shared memory is released.
+  if (qc > 0) wait_drain(smem_u32(&bars->q_full), (qc - 1) & 1);
+  for (uint32_t s = 0; s < C::KS && s < kc; ++s) {
+    const uint32_t last = kc - 1 - ((kc - 1 - s) % C::KS);
+    wait_drain(smem_u32(&bars->k_full[s]), (last / C::KS) & 1);
+  }
+}
+
+// ----------------------------------------------------------- MMA issuer --
+template <int D>
+__device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint32_t tmem) {
+  using C = Cfg<D>;
+  volatile int* abort_flag = &bars->abort;
+  volatile uint32_t* flags = bars->flags;
+  const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t sK = smem_u32(smem + C::OFF_K);
+  const uint32_t sV = smem_u32(smem + C::OFF_V);
+  constexpr uint32_t idesc_s = make_idesc_bf16(kTileQ, kTileK, 0);
+  constexpr uint32_t idesc_o = make_idesc_bf16(kTileQ, D, 1);
+  uint32_t qc = 0, kc = 0, g = 0, vc = 0, pvc = 0;
+  bool ok = true;
+
+  for (int ui = blockIdx.x; ui < p.n_units && ok; ui += gridDim.x) {
+    const Unit u = get_unit(p, ui);
+    if (u.n == 0) continue;
+    if (!wait_bounded(smem_u32(&bars->q_full), qc & 1, abort_flag, p.err, W_MMA_Q)) break;
+    ++qc;
+    tc_fence_after();
+    const uint32_t g0 = g;
+
+    // S_k = Q K_k^T into S buffer (g & 1).
+    auto issue_s = [&](int k) -> bool {
+      const uint32_t buf = g & 1;
+      if (!wait_bounded(smem_u32(&bars->s_free[buf]), ((g >> 1) & 1) ^ 1, abort_flag, p.err,
+                        W_MMA_SFREE))
+        return false;
+      const uint32_t st = kc % C::KS;
+      if (!wait_bounded(smem_u32(&bars->k_full[st]), (kc / C::KS) & 1, abort_flag, p.err, W_MMA_K))
+        return false;
+      tc_fence_after();
+      const uint32_t kbase = sK + st * C::KV_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
+        const uint64_t da = make_sdesc(sQ + (kk >> 2) * (kTileQ * 128) + off, 16, 1024);
+        const uint64_t db = make_sdesc(kbase + (kk >> 2) * (kTileK * 128) + off, 16, 1024);
+        umma_ss(tmem + buf * 64, da, db, idesc_s, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(smem_u32(&bars->k_empty[st]));
+      tc_commit(smem_u32(&bars->s_full[buf]));
+      if (k == u.n - 1) tc_commit(smem_u32(&bars->q_empty));
+      ++kc;
+      ++g;
+      return true;
+    };
+    // TMA load of V block k into the next V stage.
+    auto issue_v = [&](int k) -> bool {
+      const int kb = __ldg(p.entries + u.beg + k) >> 1;
+      const uint32_t vs = vc % C::VS;
+      if (!wait_bounded(smem_u32(&bars->v_empty[vs]), ((vc / C::VS) & 1) ^ 1, abort_flag, p.err,
+                        W_MMA_VEMPTY))
+        return false;
+      const uint32_t dst = sV + vs * C::KV_BYTES;
+      mbar_expect_tx(smem_u32(&bars->v_full[vs]), C::KV_BYTES);
+      for (int c = 0; c < C::CH; ++c)
+        tma_load_3d(dst + c * (kTileK * 128), &p.tm_v, smem_u32(&bars->v_full[vs]), c * 64,
+                    kb * kTileK, u.b * p.Hkv + u.hkv);
+      ++vc;
+      return true;
+    };
+    // Gate decision of block k (global block index g0 + k).
+    auto decision = [&](int k, bool* keep) -> bool {
+      const uint32_t gk = g0 + k;
+      if (!wait_bounded(smem_u32(&bars->dec[gk & 1]), (gk >> 1) & 1, abort_flag, p.err, W_MMA_DEC))
+        return false;
+      *keep = flags[gk & 1] != 0;
+      return true;
+    };
+
+    ok = issue_s(0) && (p.gate || issue_v(0));
+    if (ok && u.n > 1) ok = issue_s(1) && (p.gate || issue_v(1));
+    if (ok && p.gate) {
+      bool keep;
+      ok = decision(0, &keep) && (!keep || issue_v(0));
+    }
+    bool first_pv = true;
+    for (int k = 0; k < u.n && ok; ++k) {
+      const uint32_t gk = g0 + k, buf = gk & 1;
+      if (!wait_bounded(smem_u32(&bars->p_ready[buf]), (gk >> 1) & 1, abort_flag, p.err, W_MMA_P)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (flags[buf]) {
+        const uint32_t vs = pvc % C::VS;
+        if (!wait_bounded(smem_u32(&bars->v_full[vs]), (pvc / C::VS) & 1, abort_flag, p.err,
+                          W_MMA_VFULL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t vbase = sV + vs * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 16; ++kk) {
+          const uint64_t db = make_sdesc(vbase + kk * (16 * 128), kTileK * 128, 1024);
+          umma_ts(tmem + kTmemO, tmem + buf * 64 + kk * 8, db, idesc_o,
+                  (first_pv && kk == 0) ? 0u : 1u);
+        }
+        tc_commit(smem_u32(&bars->v_empty[vs]));
+        tc_commit(smem_u32(&bars->s_free[buf]));
+        tc_commit(smem_u32(&bars->o_done[pvc & 1]));
+        ++pvc;
+        first_pv = false;
+      }
+      if (p.gate && k + 1 < u.n) {
+        bool keep;
+        if (!decision(k + 1, &keep) || (keep && !issue_v(k + 1))) {
+          ok = false;
+          break;
+        }
+      }
+      if (k + 2 < u.n) {
+        if (!issue_s(k + 2) || (!p.gate && !issue_v(k + 2))) {
+          ok = false;
+          break;
+        }
+      }
+    }
+  }
+  if (!ok) {
+    // Let every MMA already issued finish, and V loads already issued land.
+    tc_commit(smem_u32(&bars->drain));
+    wait_drain(smem_u32(&bars->drain), 0);
+    for (uint32_t s = 0; s < C::VS && s < vc; ++s) {
+      const uint32_t last = vc - 1 - ((vc - 1 - s) % C::VS);
+      wait_drain(smem_u32(&bars->v_full[s]), (last / C::VS) & 1);
+    }
+  }
+}
+
+// --------------------------------------------------------------- softmax --
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Masks the logits of a partial block: x[c] = -inf for keys j = kb*64 + c
+// outside G_i (same predicate as the pattern compiler, evaluated per pair).
+__device__ __forceinline__ void mask_partial(const PrefillParams& p, int h, int i, int kb,
+                                             float (&x)[64]) {
+  const int j0 = kb * kTileK;
+  const bool row_ok = i < p.N;
+  const bool any_prim = p.window > 0 || p.n_global > 0 || p.block_local > 0 || p.n_random > 0;
+  bool rnd = false;
+  if (p.n_random > 0 && row_ok) {
+    const int nrb = (p.N + p.random_block - 1) / p.random_block;
+    const int32_t* row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
+    const int kr = j0 / p.random_block;
+    for (int r = 0; r < p.n_random; ++r) rnd |= __ldg(row + r) == kr;
+  }
+  const bool glob_row = i < p.n_global;
+  const int bl_lo = p.block_local > 0 ? (i / p.block_local) * p.block_local : 0;
+  const int bl_hi = p.block_local > 0 ? bl_lo + p.block_local : 0;
+  const int half_w = p.window / 2;
+#pragma unroll
+  for (int c = 0; c < 64; ++c) {
+    const int j = j0 + c;
+    bool v = !any_prim || glob_row || rnd || j < p.n_global;
+    if (p.window > 0) v |= p.causal ? (j > i - p.window) : (abs(i - j) <= half_w);
+    v |= (j >= bl_lo && j < bl_hi);
+    v = v && row_ok && j < p.N && (!p.causal || j <= i);
+    if (!v) x[c] = -INFINITY;
+  }
+}
+
+template <int D>
+__device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, int warp,
+                             int lane) {
+  volatile int* abort_flag = &bars->abort;
+  volatile uint32_t* flags = bars->flags;
+  const int q4 = warp & 3;              // TMEM lane quadrant of this warp
+  const int row = q4 * 32 + lane;       // query row within the tile
+  const bool leader = (warp == 2 && lane == 0);
+  const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+  uint32_t g = 0, pv_total = 0;
+
+  for (int ui = blockIdx.x; ui < p.n_units; ui += gridDim.x) {
+    const Unit u = get_unit(p, ui);
+    const int i = u.t * kTileQ + row;
+    const bool row_ok = i < p.N;
+    const int64_t orow = ((int64_t)(u.b * p.H + u.h) * p.N + i);
+    const int64_t tile_base = ((int64_t)(u.b * p.H + u.h) * p.T + u.t) * p.n_kb;
+    const float tau = (p.gate && !p.stats_only) ? __ldg(p.thresholds + u.h) : 0.f;
+    float m = -INFINITY, l = 0.f;
+    uint32_t kept = 0;
+
+    for (int k = 0; k < u.n; ++k) {
+      const uint32_t buf = g & 1;
+      const int e = __ldg(p.entries + u.beg + k);
+      const int kb = e >> 1;
+      const bool partial = e & 1;
+      if (!wait_bounded(smem_u32(&bars->s_full[buf]), (g >> 1) & 1, abort_flag, p.err, W_SM_S))
+        return;
+      tc_fence_after();
+      float x[64];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + lane_base + buf * 64, r0);
+        tmem_ld32(tmem + lane_base + buf * 64 + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[c] = __uint_as_float(r0[c]);
+          x[32 + c] = __uint_as_float(r1[c]);
+        }
+      }
+      tc_fence_before();
+      if (partial) mask_partial(p, u.h, i, kb, x);
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+
+      bool keep = true;
+      if (p.want_stats) {
+        const float wm = warp_max(mx);
+        if (lane == 0) bars->red[buf][q4] = wm;
+        named_bar_sync(kSoftmaxBar, 128);
+        const float tmax = fmaxf(fmaxf(bars->red[buf][0], bars->red[buf][1]),
+                                 fmaxf(bars->red[buf][2], bars->red[buf][3]));
+        const float stat = tmax * p.scale;
+        if (p.gate) keep = !p.stats_only && (partial || !(stat < tau));
+        if (leader) {
+          if (p.stat_out) p.stat_out[tile_base + kb] = stat;
+          if (p.mask_out) p.mask_out[tile_base + kb] = keep || p.stats_only ? 1 : 2;
+          if (p.gate) {
+            flags[buf] = keep ? 1u : 0u;
+            mbar_arrive(smem_u32(&bars->dec[buf]));
+          }
+        }
+      } else if (leader && p.mask_out) {
+        p.mask_out[tile_base + kb] = 1;
+      }
+      if (!keep) {
+        // Every thread has read S (wait::ld + fence before the barrier above).
+        if (leader) {
+          mbar_arrive(smem_u32(&bars->s_free[buf]));
+          mbar_arrive(smem_u32(&bars->p_ready[buf]));
+        }
+        ++g;
+        continue;
+      }
+
+      // Online softmax in the log2 domain with a lazily updated max.
+      const float mx2 = mx * p.scale_log2;
+      const float m_new = fmaxf(m, mx2);
+      const bool need = m_new > m + kRescaleLog2 || (m == -INFINITY && m_new != -INFINITY);
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m - m_new);   // m = -inf -> 0
+        l *= alpha;
+        m = m_new;
+      }
+      if (kept > 0 && __any_sync(0xffffffffu, need)) {
+        // O += P V of the previous kept block must be complete before O is
+        // rescaled; at most one PV is in flight here.
+        const uint32_t last = pv_total - 1;
+        if (!wait_bounded(smem_u32(&bars->o_done[last & 1]), (last >> 1) & 1, abort_flag, p.err,
+                          W_SM_O))
+          return;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          const uint32_t ta = tmem + lane_base + kTmemO + c * 32;
+          tmem_ld32(ta, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+          tmem_st32(ta, o);
+        }
+      }
+      const float mb = (m == -INFINITY) ? 0.f : m;
+      float rs = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2(fmaf(x[2 * c], p.scale_log2, -mb));
+        const float p1 = ex2(fmaf(x[2 * c + 1], p.scale_log2, -mb));
+        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l += rs;
+      tmem_st32(tmem + lane_base + buf * 64, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(kSoftmaxBar, 128);
+      if (leader) {
+        flags[buf] = 1u;
+        mbar_arrive(smem_u32(&bars->p_ready[buf]));
+      }
+      ++kept;
+      ++pv_total;
+      ++g;
+    }
+
+    if (p.stats_only) continue;
+    // Epilogue: O / l -> bf16, one row per thread.
+    uint16_t* orow_ptr = p.O + orow * D;
+    if (kept > 0) {
+      const uint32_t last = pv_total - 1;
+      if (!wait_bounded(smem_u32(&bars->o_done[last & 1]), (last >> 1) & 1, abort_flag, p.err,
+                        W_SM_EPI))
+        return;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + kTmemO + c * 32, o);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+            dst[v] = w;
+          }
+        }
+      }
+      tc_fence_before();
+    } else if (row_ok) {
+      uint4* dst = reinterpret_cast<uint4*>(orow_ptr);
+      for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+    }
+    if (row_ok && p.lse)
+      p.lse[orow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_constant__ PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + Cfg<D>::OFF_BAR);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    mbar_init(smem_u32(&bars->q_empty), 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(smem_u32(&bars->k_full[s]), 1);
+      mbar_init(smem_u32(&bars->k_empty[s]), 1);
+      mbar_init(smem_u32(&bars->v_full[s]), 1);
+      mbar_init(smem_u32(&bars->v_empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->s_full[b]), 1);
+      mbar_init(smem_u32(&bars->s_free[b]), 1);
+      mbar_init(smem_u32(&bars->p_ready[b]), 1);
+      mbar_init(smem_u32(&bars->dec[b]), 1);
+      mbar_init(smem_u32(&bars->o_done[b]), 1);
+    }
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort = 0;
+    bars->flags[0] = bars->flags[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) producer_role<D>(p, smem, bars);
+  } else if (warp == 1) {
+    if (lane == 0) mma_role<D>(p, smem, bars, tmem);
+  } else {
+    softmax_role<D>(p, bars, tmem, warp, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+int g_num_sms[64] = {0};
+bool g_attr_set[2][64] = {{false}};
+
+}  // namespace
+
+int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return set_error(SA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  if (g_num_sms[dev] == 0) {
+    e = cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_error(e, "cudaDeviceGetAttribute");
+  }
+  if (p.n_units == 0) return SA_OK;
+  const int grid = p.n_units < 2 * g_num_sms[dev] ? p.n_units : 2 * g_num_sms[dev];
+  if (d == 128) {
+    if (!g_attr_set[1][dev]) {
+      e = cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg<128>::SMEM);
+      if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute");
+      g_attr_set[1][dev] = true;
+    }
+    prefill_kernel<128><<<grid, kThreads, Cfg<128>::SMEM, stream>>>(p);
+  } else if (d == 64) {
+    if (!g_attr_set[0][dev]) {
+      e = cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg<64>::SMEM);
+      if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute");
+      g_attr_set[0][dev] = true;
+    }
+    prefill_kernel<64><<<grid, kThreads, Cfg<64>::SMEM, stream>>>(p);
+  } else {
+    return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_error(e, "prefill launch");
+  return SA_OK;
+}
+
+}  // namespace sa

@@ -1,0 +1,185 @@
+"""Seeded synthetic inputs for the five workloads (no attention arithmetic here).
+
+Shared by the tests and the benchmark, so that the CUDA path and its checks
+see the same bytes.  Everything is drawn from torch
+generators seeded as: Q = base, K = base + 1, V = base + 2, structure (unit
+directions, marked positions, random-block tables, index sets) = base + 3 ...,
+calibration draw = base + 100, with base = 1000 * workload number.  Values
+are drawn in float32 and rounded once to bf16.
+
+Workloads (names used by tests and bench):
+  tiny_static         B=1 H=H_kv=2 N=256 d=64, causal and (window 64 or globals 0..3),
+                      blocks 64x64
+  mistral_swa         B=1 H=32 H_kv=8 N=8192 d=128, causal window 4096, blocks 128x64
+  bsfa_causal         B=1 H=32 H_kv=8 N=32768 d=128, causal, block-skip rule;
+                      K = N(0,1) + 4 u_h on floor(0.02 N) marked positions per K/V head,
+                      Q = N(0,1) + 2 u_{h_kv(h)}, u_h a unit vector per K/V head
+  longformer_bigbird  B=2 H=H_kv=16 N=65536 d=64, non-causal window 512 + 64 global
+                      tokens + 3 random 64-key blocks per 64-query block
+  gather_decode       64 sequences x 1 query, H=32 H_kv=8 d=128, cache length 131072,
+                      2048 sorted unique indices per (sequence, head) = {0} and the last
+                      128 positions and 1919 uniform draws from {1 .. L-129}
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+import torch
+
+
+@dataclass
+class PrefillWorkload:
+    name: str
+    B: int
+    H: int
+    H_kv: int
+    N: int
+    d: int
+    causal: int = 0
+    window: int = 0
+    n_global: int = 0
+    block_local: int = 0
+    block_q: int = 128
+    block_k: int = 64
+    random_block: int = 64
+    n_random: int = 0
+    bsfa: bool = False
+    seed: int = 0
+    extra: dict = field(default_factory=dict)
+
+    def pattern_fields(self):
+        return dict(causal=self.causal, window=self.window, n_global=self.n_global,
+                    block_local=self.block_local, block_q=self.block_q, block_k=self.block_k,
+                    random_block=self.random_block, n_random=self.n_random)
+
+
+@dataclass
+class GatherWorkload:
+    name: str
+    S: int
+    H: int
+    H_kv: int
+    d: int
+    L: int
+    n_idx: int
+    H_idx: int
+    n_recent: int = 128
+    seed: int = 0
+
+
+WORKLOADS = {
+    "tiny_static": PrefillWorkload("tiny_static", B=1, H=2, H_kv=2, N=256, d=64, causal=1,
+                                   window=64, n_global=4, block_q=64, block_k=64, seed=1000),
+    "mistral_swa": PrefillWorkload("mistral_swa", B=1, H=32, H_kv=8, N=8192, d=128, causal=1,
+                                   window=4096, block_q=128, block_k=64, seed=2000),
+    "bsfa_causal": PrefillWorkload("bsfa_causal", B=1, H=32, H_kv=8, N=32768, d=128, causal=1,
+                                   block_q=128, block_k=64, bsfa=True, seed=3000),
+    "longformer_bigbird": PrefillWorkload("longformer_bigbird", B=2, H=16, H_kv=16, N=65536, d=64,
+                                          causal=0, window=512, n_global=64, random_block=64,
+                                          n_random=3, block_q=128, block_k=64, seed=4000),
+    "gather_decode": GatherWorkload("gather_decode", S=64, H=32, H_kv=8, d=128, L=131072,
+                                    n_idx=2048, H_idx=32, seed=5000),
+}
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def randn_bf16(shape, seed: int, device="cpu", chunk_rows: int = 1 << 22) -> torch.Tensor:
+    """N(0,1) float32 draws rounded to bf16, generated in chunks along dim 0."""
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    g = _gen(seed, device)
+    flat = out.view(shape[0], -1)
+    inner = flat.shape[1]
+    step = max(1, chunk_rows // max(inner, 1) * 64)
+    for s in range(0, shape[0], step):
+        e = min(shape[0], s + step)
+        flat[s:e] = torch.randn((e - s, inner), generator=g, device=device,
+                                dtype=torch.float32).to(torch.bfloat16)
+    return out
+
+
+def random_table(H: int, N: int, random_block: int, n_random: int, seed: int) -> np.ndarray:
+    """n_random distinct key blocks per (head, query block), uniform, ascending."""
+    nrb = -(-N // random_block)
+    n_random = min(n_random, nrb)
+    g = _gen(seed, "cpu")
+    keys = torch.rand((H, nrb, nrb), generator=g)
+    tab = keys.argsort(dim=-1)[..., :n_random].sort(dim=-1).values
+    return tab.to(torch.int32).numpy()
+
+
+def prefill_inputs(w: PrefillWorkload, device="cpu", seed: Optional[int] = None):
+    """(Q, K, V, random_table or None) for a prefill workload."""
+    base = w.seed if seed is None else seed
+    Q = randn_bf16((w.B, w.H, w.N, w.d), base, device)
+    K = randn_bf16((w.B, w.H_kv, w.N, w.d), base + 1, device)
+    V = randn_bf16((w.B, w.H_kv, w.N, w.d), base + 2, device)
+    if w.bsfa:
+        Q, K = _peaked(w, Q, K, base, device)
+    tab = None
+    if w.n_random > 0:
+        tab = random_table(w.H, w.N, w.random_block, w.n_random, base + 4)
+    return Q, K, V, tab
+
+
+def _peaked(w: PrefillWorkload, Q, K, base: int, device):
+    """K += 4 u_h on floor(0.02 N) marked positions; Q += 2 u_{h_kv(h)}."""
+    g = _gen(base + 3, "cpu")
+    u = torch.randn((w.H_kv, w.d), generator=g, dtype=torch.float32)
+    u = u / u.norm(dim=-1, keepdim=True)
+    n_mark = int(0.02 * w.N)
+    group = w.H // w.H_kv
+    Kf = K.float()
+    for hk in range(w.H_kv):
+        pos = torch.randperm(w.N, generator=g)[:n_mark].to(device)
+        Kf[:, hk, pos] += 4.0 * u[hk].to(device)
+    K = Kf.to(torch.bfloat16)
+    del Kf
+    for h in range(w.H):
+        Qh = Q[:, h].float() + 2.0 * u[h // group].to(device)
+        Q[:, h] = Qh.to(torch.bfloat16)
+    return Q, K
+
+
+def calibration_inputs(w: PrefillWorkload, device="cpu"):
+    """The calibration draw: same recipe, seed base + 100."""
+    return prefill_inputs(w, device=device, seed=w.seed + 100)
+
+
+def gather_inputs(w: GatherWorkload, device="cpu", seed: Optional[int] = None):
+    """(Q [S][H][d], K, V [S][H_kv][L][d], idx int32 [S][H_idx][n_idx]) -- idx sorted unique."""
+    base = w.seed if seed is None else seed
+    Q = randn_bf16((w.S, w.H, w.d), base, device)
+    K = randn_bf16((w.S, w.H_kv, w.L, w.d), base + 1, device)
+    V = randn_bf16((w.S, w.H_kv, w.L, w.d), base + 2, device)
+    idx = gather_index_sets(w.S, w.H_idx, w.L, w.n_idx, w.n_recent, base + 3, device)
+    return Q, K, V, idx
+
+
+def gather_index_sets(S: int, H_idx: int, L: int, n_idx: int, n_recent: int, seed: int,
+                      device="cpu", chunk: int = 64) -> torch.Tensor:
+    """{0} and {L-n_recent .. L-1} and (n_idx - n_recent - 1) distinct uniform draws
+    from {1 .. L-n_recent-1}, sorted ascending, per (sequence, index head)."""
+    n_recent = min(n_recent, L - 1)
+    n_draw = n_idx - n_recent - 1
+    pool = L - n_recent - 1
+    assert 0 <= n_draw <= pool, "index set larger than the cache"
+    g = _gen(seed, device)
+    rows = S * H_idx
+    out = torch.empty((rows, n_idx), dtype=torch.int32, device=device)
+    fixed = torch.cat([torch.zeros(1, dtype=torch.int64, device=device),
+                       torch.arange(L - n_recent, L, device=device)])
+    for s in range(0, rows, chunk):
+        e = min(rows, s + chunk)
+        keys = torch.rand((e - s, pool), generator=g, device=device)
+        draw = keys.topk(n_draw, dim=1).indices + 1 if n_draw > 0 else \
+            torch.empty((e - s, 0), dtype=torch.int64, device=device)
+        allv = torch.cat([fixed.expand(e - s, -1), draw], dim=1)
+        out[s:e] = allv.sort(dim=1).values.to(torch.int32)
+    return out.view(S, H_idx, n_idx)

@@ -1,0 +1,204 @@
+/*
+ * sparse_attn.h -- C ABI of the B200 (sm_100a) block-sparse attention library.
+ *
+ * The operation (web pages on sparse attention):
+ *   "Sparse Attention Weights Assumption" (1cademy), sparse attention output
+ *   formula:  out_i = sum_{j in G_i} alpha'_{i,j} v_j,  G_i subset of {0..i}
+ *   (causal).  alpha' is the softmax of the scaled logits s_ij = scale*q_i.k_j
+ *   taken over G_i only, so a full G_i gives the glossary's dense
+ *   softmax(Q K^T / sqrt(d_k)) V ("sparse attention mechanism" glossary,
+ *   chipfoundryservices, "Standard Attention Bottleneck").
+ *
+ * G_i comes from one of two places:
+ *   - sparse_attn_prefill*: a static pattern (sa_pattern_t) -- the union, by
+ *     logical OR ("SAS: Sparse Attention Synthesizer", kindchill, Step 5,
+ *     component 2), of a sliding window, global tokens, block-local blocks and
+ *     BigBird-style random blocks (glossary, "Sparse Attention Patterns" table
+ *     and "Mistral/Mixtral Sliding Window Attention"), intersected with the
+ *     causal constraint -- optionally pruned by the dynamic Block-Sparse-
+ *     FlashAttention rule ("Block Sparse Flash Attention", montaan AI Radio,
+ *     paper summary and improvements): the exact QK^T tile of a 64-key block is
+ *     computed, its maximum scaled logit is compared with a per-head calibrated
+ *     threshold, and below it the block's V load and PV product are skipped and
+ *     its keys leave G_i for every row of the 128-row query tile.
+ *   - sparse_attn_gather: explicit, sorted index sets over a KV cache (decode).
+ *
+ * K/V heads are shared by contiguous groups of query heads (GQA/MQA, glossary
+ * "Multi-Query and Grouped-Query Attention"): h_kv = h / (H / H_kv).
+ *
+ * Conventions for every call below.
+ *   - Tensors are caller-owned, device-resident, contiguous row-major bf16
+ *     (raw IEEE bfloat16 bit patterns, passed as void*), 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronise, except where a comment says so.
+ *   - Return value: SA_OK or an SA_ERR_* code; sparse_attn_last_error() then
+ *     gives a message (thread-local).  Argument errors are detected on the host
+ *     before anything is launched.
+ *   - Errors found by a kernel while it runs (an index out of range in a
+ *     gather set, a pipeline wait that ran out of time) are recorded in a
+ *     device error word instead of faulting; read and clear it with
+ *     sparse_attn_check_device_error().
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st *sa_stream_t;
+
+enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,   /* bad pointer, shape, alignment or descriptor           */
+    SA_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for            */
+    SA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed                      */
+    SA_ERR_NO_MEMORY = 4,     /* host or device allocation failed                      */
+    SA_ERR_TIMEOUT = 5,       /* device: a pipeline wait ran out of time; kernel bailed */
+    SA_ERR_DEVICE_INDEX = 6   /* device: a gather index was outside [0, L); row skipped */
+};
+
+/*
+ * Static pattern descriptor.  G_i = { j < N : base(i, j) and (!causal or j <= i) }
+ * where base is the logical OR of the primitives that are on (all keys when
+ * none is on):
+ *   window       W > 0.  causal: j in [i-W+1, i]  (Mistral rule, glossary);
+ *                non-causal: |i - j| <= W/2 ("w nearest neighbours").
+ *   n_global     g > 0.  i < g or j < g: tokens 0..g-1 see every key and are
+ *                seen by every query (1cademy "Global Tokens in Attention").
+ *   block_local  b > 0.  i / b == j / b (glossary "Blockwise").
+ *   random       n_random > 0 and random_table != NULL: key j is visible from
+ *                query i when j / random_block is listed in
+ *                random_table[h][i / random_block][0 .. n_random) (BigBird).
+ * block_q x block_k is the tile of the block-skip rule and of the block FLOP
+ * accounting.  The kernels tile 128 query rows x 64 keys, so block_k must be 64
+ * and block_q 64 or 128 (128 when the block-skip rule is used).
+ * scale: logit scale; 0 means 1/sqrt(d).
+ */
+typedef struct {
+    int32_t causal;
+    int32_t window;
+    int32_t n_global;
+    int32_t block_local;
+    int32_t block_q;
+    int32_t block_k;
+    int32_t random_block;          /* multiple of 64 when random blocks are on            */
+    int32_t n_random;
+    const int32_t *random_table;   /* HOST pointer, int32 [H][ceil(N/random_block)][n_random],
+                                      entries in [0, ceil(N/random_block)); read only while
+                                      a plan is created (the plan keeps a device copy)    */
+    const float *thresholds;       /* DEVICE pointer, float [H] block-skip thresholds in
+                                      scaled-logit (natural-log) units, or NULL = rule off.
+                                      Used by sparse_attn_prefill only; plans take the
+                                      thresholds per call.                                */
+    float scale;
+} sa_pattern_t;
+
+/* A compiled pattern: per-(head, 128-row query tile) lists of 64-key blocks
+ * with a full/partial flag, a longest-first work order and a device copy of the
+ * random table.  Owns device memory; freed by sparse_attn_plan_destroy. */
+typedef struct sa_plan sa_plan_t;
+
+typedef struct {
+    int32_t T_q;            /* 128-row query tiles per (b, h): ceil(N/128)              */
+    int32_t n_kb;           /* 64-key blocks per row: ceil(N/64)                         */
+    int64_t n_units;        /* work units B*H*T_q                                        */
+    int64_t blocks;         /* listed (tile, key block) pairs over all (b, h), 128x64   */
+    int64_t blocks_full;    /* ... of which every pair is in G (may be skipped)         */
+    int64_t blocks_desc;    /* listed blocks at the descriptor's block_q x block_k      */
+    int64_t pairs;          /* sum over (b, h, i) of |G_i| of the static pattern        */
+    double compile_ms;      /* host time spent compiling the pattern                    */
+} sa_plan_info_t;
+
+/* Compile `pat` for Q [B][H][N][d], K/V [B][H_kv][N][d].  Host work plus
+ * cudaMalloc/cudaMemcpy on the current device; synchronous.  Errors:
+ * SA_ERR_INVALID_ARG (shapes, H % H_kv != 0, bad descriptor or table entry),
+ * SA_ERR_UNSUPPORTED (d not 64/128, block_k != 64, random_block % 64 != 0),
+ * SA_ERR_NO_MEMORY, SA_ERR_CUDA.  On success *out owns the plan. */
+int sparse_attn_plan_create(const sa_pattern_t *pat, int B, int H, int H_kv, int N, int d,
+                            sa_plan_t **out);
+int sparse_attn_plan_info(const sa_plan_t *plan, sa_plan_info_t *info);
+void sparse_attn_plan_destroy(sa_plan_t *plan);   /* synchronises the device; NULL ok */
+
+/* Prefill with a compiled plan.
+ *   Q [B][H][N][d], K, V [B][H_kv][N][d] (bf16, device, read); O [B][H][N][d]
+ *   (bf16, device, written).
+ *   thresholds: device float [H] (block-skip rule on) or NULL (static pattern only).
+ *   lse_out: device float [B][H][N] = ln sum_{j in G_i} exp(s_ij), -inf for an
+ *            empty G_i; or NULL.
+ *   block_mask_out: device uint8 [B][H][T_q][n_kb]; 0 = block not listed,
+ *            1 = computed and kept, 2 = skipped by the rule; or NULL.
+ *   block_stat_out: device float [B][H][T_q][n_kb]; for listed blocks the
+ *            maximum scaled logit over the tile's visible pairs (unlisted
+ *            entries are left untouched); or NULL.
+ * The plan must not be destroyed while a launch that uses it may still run. */
+int sparse_attn_prefill_plan(const sa_plan_t *plan, const void *Q, const void *K,
+                             const void *V, void *O, const float *thresholds,
+                             float *lse_out, uint8_t *block_mask_out,
+                             float *block_stat_out, sa_stream_t stream);
+
+/* One-shot prefill: looks the pattern up in a per-process plan cache (keyed on
+ * every descriptor field, the random table's contents and the shapes), compiles
+ * it on a miss (synchronous, see sparse_attn_plan_create), then launches as
+ * sparse_attn_prefill_plan with pat->thresholds. */
+int sparse_attn_prefill(const void *Q, const void *K, const void *V, void *O,
+                        int B, int H, int H_kv, int N, int d, const sa_pattern_t *pat,
+                        float *lse_out, uint8_t *block_mask_out, sa_stream_t stream);
+
+/* Block-statistics pass of the block-skip rule over a plan: computes the
+ * QK^T tiles of every listed block and writes block_stat_out (layout as
+ * above) and block_mask_out (1 for every listed block); no V is read and no
+ * output is written.  Used to calibrate thresholds on a calibration draw. */
+int sparse_attn_block_stats(const sa_plan_t *plan, const void *Q, const void *K,
+                            float *block_stat_out, uint8_t *block_mask_out,
+                            sa_stream_t stream);
+
+/* Per-head threshold calibration from a statistics pass: for each head h,
+ * thresholds_out[h] = the element of rank floor((n_h - 1) * q) (0-based,
+ * ascending) among the statistics of head h's FULL blocks over all b and
+ * tiles, n_h their number (q = 0.5 gives the lower median).  block_stat is
+ * the output of sparse_attn_block_stats for the same plan.  Device float [H]
+ * out; -inf when a head has no full block. */
+int sparse_attn_calibrate(const sa_plan_t *plan, const float *block_stat, double q,
+                          float *thresholds_out, sa_stream_t stream);
+
+/* Explicit index-set attention over a KV cache (decode, one query per sequence).
+ *   Q [S][H][d] bf16; K, V [S][H_kv][L][d] bf16; O [S][H][d] bf16 (written).
+ *   idx: device int32 [S][H_idx][n_idx]; each set sorted ascending, unique, in
+ *        [0, L).  H_idx == H: one set per query head; H_idx == H_kv: one set per
+ *        K/V head, shared by its query heads.
+ *   idx_len: device int32 [S][H_idx] (entries used, 0..n_idx) or NULL (= n_idx).
+ *   lse_out: device float [S][H] or NULL.
+ *   An empty set gives O = 0, lse = -inf.  An index outside [0, L) is skipped
+ *   and recorded as SA_ERR_DEVICE_INDEX in the device error word. */
+int sparse_attn_gather(const void *Q, const void *K, const void *V, const int32_t *idx,
+                       const int32_t *idx_len, void *O, int S, int H, int H_kv, int H_idx,
+                       int L, int n_idx, int d, float scale, float *lse_out,
+                       sa_stream_t stream);
+
+/* Host-only pattern compiler (no GPU needed): the block lists a plan holds, at
+ * tile_q x tile_k granularity.  H_pat = H when random blocks are on, else 1
+ * (the lists do not depend on the head).  First call with row_ptr == NULL to
+ * get *H_pat_out, *T_out, *n_entries_out; then call again with
+ * row_ptr int32 [H_pat*T + 1], kb int32 [n_entries], full uint8 [n_entries]
+ * and, optionally, cnt int64 [n_entries] (visible pairs per listed block). */
+int sparse_attn_compile_pattern(const sa_pattern_t *pat, int H, int N, int tile_q,
+                                int tile_k, int *H_pat_out, int *T_out,
+                                int64_t *n_entries_out, int32_t *row_ptr, int32_t *kb,
+                                uint8_t *full, int64_t *cnt);
+
+/* Waits for `stream`, then reads and clears the device error word.  Returns
+ * SA_OK, SA_ERR_TIMEOUT, SA_ERR_DEVICE_INDEX or SA_ERR_CUDA. */
+int sparse_attn_check_device_error(sa_stream_t stream);
+
+/* Message for the last error on this thread ("" if none). */
+const char *sparse_attn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPARSE_ATTN_H */

@@ -1,0 +1,89 @@
+"""The C-ABI library loads, exports every function include/sparse_attn.h declares,
+and rejects bad arguments on the host before any launch (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "sparse_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparse_attn_\w+)\s*\(", src)))
+
+
+def test_header_and_binding_agree(product):
+    assert _declared() == sorted(product.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(product):
+    lib = ctypes.CDLL(product.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_library_is_sm100a_only(product):
+    """The shared library carries sm_100a code (built with -gencode arch=compute_100a,code=sm_100a)."""
+    import subprocess
+    out = subprocess.run(["cuobjdump", "--list-elf", product.LIB_PATH], capture_output=True,
+                         text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    archs = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert archs == {"100a"}, archs
+
+
+def _err(product, rc):
+    return rc, product._lib.lib().sparse_attn_last_error().decode()
+
+
+def test_argument_errors_on_host(product):
+    L = product._lib.lib()
+    pat, _t = product.Pattern(causal=1).to_c()
+    h = ctypes.c_void_p()
+    # H not a multiple of H_kv
+    rc, msg = _err(product, L.sparse_attn_plan_create(ctypes.byref(pat), 1, 6, 4, 128, 128,
+                                                      ctypes.byref(h)))
+    assert rc == product.SA_ERR_INVALID_ARG and "multiple" in msg
+    # unsupported head dim
+    rc, msg = _err(product, L.sparse_attn_plan_create(ctypes.byref(pat), 1, 4, 4, 128, 96,
+                                                      ctypes.byref(h)))
+    assert rc == product.SA_ERR_UNSUPPORTED
+    # unsupported block_k
+    pat2, _t2 = product.Pattern(causal=1, block_k=32).to_c()
+    rc, _ = _err(product, L.sparse_attn_plan_create(ctypes.byref(pat2), 1, 4, 4, 128, 64,
+                                                    ctypes.byref(h)))
+    assert rc == product.SA_ERR_UNSUPPORTED
+    # null tensors to the gather entry
+    rc, _ = _err(product, L.sparse_attn_gather(None, None, None, None, None, None, 1, 4, 4, 4,
+                                               16, 4, 64, 0.0, None, None))
+    assert rc == product.SA_ERR_INVALID_ARG
+    # misaligned pointer
+    rc, msg = _err(product, L.sparse_attn_gather(8, 16, 16, 16, None, 16, 1, 4, 4, 4, 16, 4, 64,
+                                                 0.0, None, None))
+    assert rc == product.SA_ERR_INVALID_ARG and "aligned" in msg
+    # bad H_idx
+    rc, _ = _err(product, L.sparse_attn_gather(16, 16, 16, 16, None, 16, 1, 4, 2, 3, 16, 4, 64,
+                                               0.0, None, None))
+    assert rc == product.SA_ERR_INVALID_ARG
+
+
+def test_random_table_out_of_range_is_rejected(product):
+    import numpy as np
+    tab = np.full((1, 2, 1), 5, np.int32)   # only 2 blocks exist for N=128
+    with pytest.raises(product.SparseAttnError) as e:
+        product.compile_pattern(product.Pattern(n_random=1, random_block=64, random_table=tab), 1, 128)
+    assert e.value.code == product.SA_ERR_INVALID_ARG
+
+
+def test_no_oracle_in_product_path():
+    """The product package never imports, loads or names the oracle."""
+    pkg = os.path.join(ROOT, "block_sparse_attention_29_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"\boracle\b|sa_oracle", src), f

@@ -1,0 +1,162 @@
+"""The fused block-skip rule on the GPU against the fp64 oracle.
+
+Block masks must be identical to the oracle's except for blocks whose oracle
+statistic lies within 1e-3 of the threshold; those are counted and their rows
+are checked against the oracle replaying the GPU's decisions.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_29_b200.workloads import (WORKLOADS, calibration_inputs,
+                                                      prefill_inputs)
+
+from _parity import NEAR_BAND, assert_close, compare_masks
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(N=1024, H=4, Hkv=2, d=128):
+    return dataclasses.replace(WORKLOADS["bsfa_causal"], N=N, H=H, H_kv=Hkv, d=d)
+
+
+def _tensors(w, device):
+    Q, K, V, _ = prefill_inputs(w, device="cpu")
+    return Q.to(device), K.to(device), V.to(device)
+
+
+@pytest.mark.parametrize("d", [128, 64])
+def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d):
+    w = _small(d=d)
+    Qc, Kc, Vc, _ = calibration_inputs(w, device="cpu")
+    opat = oracle_mod.Pattern(**w.pattern_fields())
+    full_c, stat_c, _ = oracle_mod.block_stats(opat, Qc, Kc)
+    # the kernel compares fp32 statistics with fp32 thresholds: give the oracle
+    # the same (rounded) threshold values
+    tau = oracle_mod.calibrate_thresholds(full_c, stat_c).astype(np.float32).astype(np.float64)
+    Q, K, V = _tensors(w, cuda)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    tau_d = torch.tensor(tau, dtype=torch.float32, device=cuda)
+    mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
+    stat = torch.full((w.B, w.H, plan.T, plan.n_kb), float("-inf"), device=cuda)
+    lse = torch.empty((w.B, w.H, w.N), device=cuda)
+    O = plan.prefill(Q, K, V, thresholds=tau_d, lse=lse, block_mask=mask, block_stat=stat)
+    product.check_device_error()
+
+    Or, lr, om, ost, ofull = oracle_mod.prefill(opat, Q.cpu(), K.cpu(), V.cpu(),
+                                                thresholds=tau, want_blocks=True)
+    n, n_near, override = compare_masks(mask.cpu().numpy(), om, ost, tau)
+    listed = om != 0
+    assert np.abs(stat.cpu().numpy()[listed] - ost[listed]).max() < 1e-3
+    skipped = (om == 2).sum() / max(1, ofull.sum())
+    assert 0.2 < skipped < 0.8, f"skip fraction {skipped}"
+    if n_near:
+        Or, lr = oracle_mod.prefill(opat, Q.cpu(), K.cpu(), V.cpu(), thresholds=tau,
+                                    override=override)
+    assert_close(O, Or)
+    assert_close(lse, lr, what="lse")
+
+
+def test_bsfa_extreme_thresholds(product, oracle_mod, cuda):
+    w = _small(N=768, H=2, Hkv=1)
+    Q, K, V = _tensors(w, cuda)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
+    # -inf: nothing skipped, equals the static causal path bit for bit
+    O_static = plan.prefill(Q, K, V)
+    O_minf = plan.prefill(Q, K, V, thresholds=torch.full((w.H,), float("-inf"), device=cuda),
+                          block_mask=mask)
+    torch.cuda.synchronize()
+    assert torch.equal(O_static, O_minf)
+    assert not (mask == 2).any()
+    # +inf: every full block skipped; equals the diagonal-only static pattern
+    O_pinf = plan.prefill(Q, K, V, thresholds=torch.full((w.H,), float("inf"), device=cuda),
+                          block_mask=mask)
+    product.check_device_error()
+    _, _, _, _, full = oracle_mod.prefill(oracle_mod.Pattern(**w.pattern_fields()), Q.cpu(),
+                                          K.cpu(), V.cpu(), rows=np.array([[0, 0, 0]]),
+                                          want_blocks=True)
+    row_ptr, kb, fl, cnt, _, T = product.compile_pattern(product.Pattern(**w.pattern_fields()),
+                                                         w.H, w.N)
+    m = mask.cpu().numpy()
+    for t in range(T):
+        ks = kb[row_ptr[t]:row_ptr[t + 1]]
+        fs = fl[row_ptr[t]:row_ptr[t + 1]]
+        assert (m[0, :, t, ks[fs]] == 2).all() and (m[0, :, t, ks[~fs]] == 1).all()
+    diag = oracle_mod.Pattern(causal=1, block_local=128)
+    Or, _ = oracle_mod.prefill(diag, Q.cpu(), K.cpu(), V.cpu())
+    assert_close(O_pinf, Or)
+
+
+def test_device_calibration_matches_oracle(product, oracle_mod, cuda):
+    """Statistics pass + per-head rank selection on the GPU == oracle calibration."""
+    w = _small(N=1024, H=4, Hkv=2)
+    Qc, Kc, _, _ = calibration_inputs(w, device="cpu")
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    stat = plan.block_stats(Qc.to(cuda), Kc.to(cuda))
+    tau_gpu = plan.calibrate(stat, 0.5).cpu().numpy()
+    opat = oracle_mod.Pattern(**w.pattern_fields())
+    full, ostat, _ = oracle_mod.block_stats(opat, Qc, Kc)
+    tau = oracle_mod.calibrate_thresholds(full, ostat)
+    assert np.abs(tau_gpu - tau).max() < 1e-3
+    # the GPU selection is exact on its own statistics
+    s = stat.cpu().numpy()
+    for h in range(w.H):
+        v = np.sort(s[:, h][full[:, h]])
+        assert tau_gpu[h] == np.float32(v[(len(v) - 1) // 2])
+        assert tau_gpu[h] == np.float32(v[(len(v) - 1) // 2])
+
+
+@pytest.mark.slow
+def test_bsfa_full_size_sampled(product, oracle_mod, cuda):
+    """bsfa_causal at N=32768: device calibration on the calibration draw, then the
+    rule; masks checked on sampled tiles, outputs on sampled rows."""
+    w = WORKLOADS["bsfa_causal"]
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    Qc, Kc, _, _ = calibration_inputs(w, device=cuda)
+    tau_d = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
+    del Qc, Kc
+    Q, K, V, _ = prefill_inputs(w, device=cuda)
+    mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
+    stat = torch.empty((w.B, w.H, plan.T, plan.n_kb), device=cuda)
+    O = plan.prefill(Q, K, V, thresholds=tau_d, block_mask=mask, block_stat=stat)
+    product.check_device_error()
+    tau = tau_d.cpu().numpy().astype(np.float64)
+    m = mask.cpu().numpy()
+    s = stat.cpu().numpy()
+    # property over every block: the decision is the rule applied to the GPU statistic
+    row_ptr, kb, fl, cnt, _, T = product.compile_pattern(product.Pattern(**w.pattern_fields()),
+                                                         w.H, w.N)
+    full = np.zeros((plan.T, plan.n_kb), bool)
+    for t in range(T):
+        full[t, kb[row_ptr[t]:row_ptr[t + 1]][fl[row_ptr[t]:row_ptr[t + 1]]]] = True
+    skip_expected = full[None, None] & (s < tau.reshape(1, -1, 1, 1).astype(np.float32))
+    assert np.array_equal(m == 2, skip_expected)
+    frac = (m == 2).sum() / (full.sum() * w.H)
+    assert 0.35 < frac < 0.65, frac
+    # oracle on sampled tiles: statistics and decisions
+    g = np.random.default_rng(5)
+    tiles = [(0, h, t) for h in (0, w.H - 1) for t in (0, 1, T // 2, T - 1)]
+    tiles += [(0, int(g.integers(w.H)), int(g.integers(T))) for _ in range(8)]
+    opat = oracle_mod.Pattern(**w.pattern_fields())
+    Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
+    rows, override = [], np.full(m.shape, -1, np.int8)
+    near_total = 0
+    for (b, h, t) in tiles:
+        ocnt, ofull, ostat, omask = oracle_mod.tile_blocks(opat, Qh, Kh, b, h, t, thresholds=tau)
+        lst = omask != 0
+        assert np.array_equal(m[b, h, t] != 0, lst)
+        assert np.abs(s[b, h, t][lst] - ostat[lst]).max() < 1e-3
+        diff = (m[b, h, t] != omask)
+        near = np.abs(ostat - tau[h]) <= NEAR_BAND
+        assert not (diff & ~near).any()
+        near_total += int(diff.sum())
+        override[b, h, t][diff] = (m[b, h, t][diff] == 2)
+        for i in (t * 128, t * 128 + 63, t * 128 + 127):
+            rows.append((b, h, i))
+    rows = np.array(rows, np.int32)
+    Or, _ = oracle_mod.prefill(opat, Qh, Kh, Vh, thresholds=tau, rows=rows, override=override)
+    sel = tuple(torch.from_numpy(rows[:, k]).long() for k in range(3))
+    assert_close(O.cpu()[sel], Or)
