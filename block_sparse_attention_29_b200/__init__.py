@@ -26,7 +26,8 @@ import numpy as np
 from ._lib import (EXPORTS, LIB_PATH, SA_ERR_DEVICE_INDEX, SA_ERR_INVALID_ARG, SA_ERR_TIMEOUT,
                    SA_ERR_UNSUPPORTED, SA_OK, SaPattern, SaPlanInfo, SparseAttnError, check, lib)
 
-__all__ = ["Pattern", "Plan", "sparse_attn_prefill", "sparse_attn_gather", "compile_pattern",
+__all__ = ["Pattern", "Plan", "sparse_attn_prefill", "sparse_attn_prefill_noalloc",
+           "sparse_attn_gather", "compile_pattern",
            "check_device_error", "SparseAttnError", "EXPORTS", "LIB_PATH", "SA_OK",
            "SA_ERR_INVALID_ARG", "SA_ERR_UNSUPPORTED", "SA_ERR_TIMEOUT", "SA_ERR_DEVICE_INDEX"]
 
@@ -170,6 +171,28 @@ def sparse_attn_prefill(Q, K, V, pattern: Pattern, thresholds=None, O=None, lse=
     check(lib().sparse_attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), B, H, Hkv, N, d,
                                     ctypes.byref(st), _ptr(lse), _ptr(block_mask),
                                     _stream(stream)))
+    return O
+
+
+def sparse_attn_prefill_noalloc(Q, K, V, pattern: Pattern, O, thresholds=None, lse=None,
+                                stream=None):
+    """Prefill through the entry point that allocates no device memory: for
+    callers that cannot call cudaMalloc at run time (external pools or
+    allocation-free inference runtimes).  The caller supplies O (and lse);
+    the library copies the compiled pattern into its fixed 8 MiB static device
+    array.  Calls that may overlap on the GPU share that array and race."""
+    import torch
+    B, H, N, d = Q.shape
+    Hkv = K.shape[1]
+    _check_tensor("Q", Q, (B, H, N, d), torch.bfloat16)
+    _check_tensor("K", K, (B, Hkv, N, d), torch.bfloat16)
+    _check_tensor("V", V, (B, Hkv, N, d), torch.bfloat16)
+    _check_tensor("O", O, (B, H, N, d), torch.bfloat16)
+    if lse is not None:
+        _check_tensor("lse", lse, (B, H, N), torch.float32)
+    st, _tab = pattern.to_c(_ptr(thresholds) or 0)
+    check(lib().sparse_attn_prefill_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), B, H, Hkv, N, d,
+                                            ctypes.byref(st), _ptr(lse), _stream(stream)))
     return O
 
 

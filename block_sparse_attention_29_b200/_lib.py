@@ -25,7 +25,7 @@ EXPORTS = (
     "sparse_attn_plan_create", "sparse_attn_plan_info", "sparse_attn_plan_destroy",
     "sparse_attn_prefill_plan", "sparse_attn_prefill", "sparse_attn_block_stats",
     "sparse_attn_calibrate", "sparse_attn_gather", "sparse_attn_compile_pattern",
-    "sparse_attn_check_device_error", "sparse_attn_last_error",
+    "sparse_attn_check_device_error", "sparse_attn_last_error", "sparse_attn_prefill_noalloc",
 )
 
 
@@ -73,6 +73,8 @@ def lib():
         L.sparse_attn_plan_destroy.restype = None
         L.sparse_attn_prefill_plan.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.sparse_attn_prefill.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, P, vp, vp, vp]
+        L.sparse_attn_prefill_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, P, vp,
+                                                  vp]
         L.sparse_attn_block_stats.argtypes = [vp, vp, vp, vp, vp, vp]
         L.sparse_attn_calibrate.argtypes = [vp, vp, f64, vp, vp]
         L.sparse_attn_gather.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,

@@ -77,6 +77,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_current_device(int want) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+  if (dev != want)
+    return set_error(SA_ERR_INVALID_ARG, "plan was created on device %d, current device is %d",
+                     want, dev);
+  return SA_OK;
+}
+}  // namespace
+
 // 3-D bf16 map over a [BH][N][d] tensor, box {64, rows, 1}, 128-byte swizzle.
 // Rows past N read as zero.
 int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows) {
@@ -92,19 +105,6 @@ int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows) 
   if (r != CUDA_SUCCESS) return set_error(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return SA_OK;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int check_current_device(int want) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
-  if (dev != want)
-    return set_error(SA_ERR_INVALID_ARG, "plan was created on device %d, current device is %d",
-                     want, dev);
-  return SA_OK;
-}
-}  // namespace
 
 }  // namespace sa
 

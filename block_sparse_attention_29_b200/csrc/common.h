@@ -60,6 +60,10 @@ struct PrefillParams {
 
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
 
+// 3-D bf16 TMA map over a [BH][N][d] tensor, box {64, rows, 1}, 128-byte
+// swizzle; rows past N read as zero.
+int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows);
+
 // ----------------------------------------------------------------- gather --
 struct GatherParams {
   const uint16_t* Q;   // [S][H][d]

@@ -180,6 +180,24 @@ int sparse_attn_gather(const void *Q, const void *K, const void *V, const int32_
                        int L, int n_idx, int d, float scale, float *lse_out,
                        sa_stream_t stream);
 
+/* Prefill that allocates no device memory.  (The pages have no counterpart:
+ * this is a deployment variant of sparse_attn_prefill.)  For callers that
+ * cannot call cudaMalloc at run time -- code whose device memory is owned by
+ * an external pool or allocator, or runtimes that forbid allocation on the
+ * inference path.  Same arguments and result as sparse_attn_prefill (block
+ * mask output excepted); the compiled pattern is not cached but rebuilt on the
+ * host each call and copied into a fixed 8 MiB static device array that the
+ * library holds on every device until the process exits.  Patterns whose
+ * block lists, work order and random table need more than 8 MiB are rejected
+ * with SA_ERR_INVALID_ARG.  The first call on a device looks up the array's
+ * device address (with that device current); make it before any stream
+ * capture.  Every call reuses the array: calls that can overlap on the GPU
+ * (different streams without ordering) race; calls on one stream do not.
+ * Calls no cudaMalloc, cudaFree or other allocating library routine. */
+int sparse_attn_prefill_noalloc(const void *Q, const void *K, const void *V, void *O,
+                                int B, int H, int H_kv, int N, int d, const sa_pattern_t *pat,
+                                float *lse_out, sa_stream_t stream);
+
 /* Host-only pattern compiler (no GPU needed): the block lists a plan holds, at
  * tile_q x tile_k granularity.  H_pat = H when random blocks are on, else 1
  * (the lists do not depend on the head).  First call with row_ptr == NULL to
