@@ -118,6 +118,7 @@ struct sa_plan {
   int32_t* d_entries = nullptr;
   int32_t* d_units = nullptr;
   int32_t* d_rtab = nullptr;
+  int* d_sched = nullptr;      // work-queue counters, zero between launches
   sa_plan_info_t info{};
 };
 
@@ -135,6 +136,7 @@ void plan_free(sa_plan_t* p) {
   cudaFree(p->d_entries);
   cudaFree(p->d_units);
   cudaFree(p->d_rtab);
+  cudaFree(p->d_sched);
   if (prev >= 0 && prev != p->device) cudaSetDevice(prev);
   delete p;
 }
@@ -210,6 +212,7 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
   p->row_ptr = plan->d_row_ptr;
   p->entries = plan->d_entries;
   p->units = plan->d_units;
+  p->sched = plan->d_sched;
   p->rtab = plan->d_rtab;
   p->thresholds = thresholds;
   p->n_units = plan->n_units;
@@ -312,33 +315,17 @@ int sparse_attn_plan_create(const sa_pattern_t* pat, int B, int H, int H_kv, int
     plan->info.blocks_desc = int64_t(cd.kb.size()) * int64_t(B) * (cd.H_pat == 1 ? H : 1);
   }
 
-  // Work order: longest list first; ties by tile, then (b, kv head, head) so
-  // the query heads that share K/V blocks run next to each other.
-  const int T = cp.T;
-  plan->n_units = B * H * T;
-  std::vector<int32_t> units(plan->n_units);
-  std::iota(units.begin(), units.end(), 0);
-  auto cost = [&](int32_t u) {
-    const int t = u % T, h = (u / T) % H;
-    const int row = (cp.H_pat > 1 ? h : 0) * T + t;
-    return cp.row_ptr[row + 1] - cp.row_ptr[row];
-  };
-  const int group = H / H_kv;
-  std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
-    const int ca = cost(a), cb = cost(b);
-    if (ca != cb) return ca > cb;
-    const int ta = a % T, tb = b % T;
-    if (ta != tb) return ta < tb;
-    const int bha = a / T, bhb = b / T;
-    const int ba = bha / H, bb = bhb / H, ha = bha % H, hb = bhb % H;
-    if (ba != bb) return ba < bb;
-    if (ha / group != hb / group) return ha / group < hb / group;
-    return ha < hb;
-  });
+  plan->n_units = B * cp.T * H;
+  std::vector<int32_t> units;
+  order_units(cp, B, H, H_kv, &units);
 
   rc = upload(&plan->d_row_ptr, cp.row_ptr.data(), cp.row_ptr.size());
   if (!rc) rc = upload(&plan->d_entries, entries.data(), entries.size());
   if (!rc) rc = upload(&plan->d_units, units.data(), units.size());
+  if (!rc) {
+    const int zeros[2] = {0, 0};
+    rc = upload(&plan->d_sched, zeros, 2);
+  }
   if (!rc && pat->n_random > 0 && pat->random_table) {
     const int nrb = (N + pat->random_block - 1) / pat->random_block;
     rc = upload(&plan->d_rtab, pat->random_table, size_t(H) * nrb * pat->n_random);

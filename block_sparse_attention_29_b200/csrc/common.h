@@ -45,6 +45,8 @@ struct PrefillParams {
   const int32_t* row_ptr;   // [H_pat*T + 1]
   const int32_t* entries;   // block lists
   const int32_t* units;     // work order: unit = (b*H + h)*T + t
+  int* sched;               // [2] work-queue counters (next unit, CTAs done); zero
+                            // between launches (the last CTA of a launch resets them)
   const int32_t* rtab;      // random table [H][n_rb][n_random] or null
   const float* thresholds;  // [H] or null
   int n_units;
@@ -99,5 +101,8 @@ int compile_pattern(const sa_pattern_t* pat, int H, int N, int tile_q, int tile_
                     CompiledPattern* out);
 // Validates the descriptor fields that do not depend on the kernel.
 int validate_pattern(const sa_pattern_t* pat, int H, int N);
+// Work order of the B*H*T units (unit = (b*H + h)*T + t): longest first in
+// coarse cost buckets, tile-major with GQA siblings adjacent inside a bucket.
+void order_units(const CompiledPattern& cp, int B, int H, int H_kv, std::vector<int32_t>* units);
 
 }  // namespace sa

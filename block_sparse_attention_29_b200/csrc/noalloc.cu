@@ -18,9 +18,11 @@
 // call before any stream capture begins.
 //
 // Sharing: every call uses the same array and leaves the last call's contents
-// in it.  The plan data is rewritten in full by each call, so nothing needs to
-// start at zero.  Calls whose copies and kernels may overlap on the GPU (for
-// example on two streams without ordering between them) race on the array.
+// in it.  The plan data is rewritten in full by each call; the two work-queue
+// counters at the start of the array must start at zero and are cleared by
+// each call before its launch.  Calls whose copies and kernels may overlap on
+// the GPU (for example on two streams without ordering between them) race on
+// the array.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -96,7 +98,8 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   const size_t b_ent = round256(std::max<size_t>(cp.kb.size(), 1) * 4);
   const size_t b_units = round256(size_t(n_units) * 4);
   const size_t b_rtab = rnd ? round256(size_t(H) * nrb * pat->n_random * 4) : 0;
-  const size_t need = b_row + b_ent + b_units + b_rtab;
+  const size_t b_sched = 256;   // work-queue counters
+  const size_t need = b_sched + b_row + b_ent + b_units + b_rtab;
   if (need > kNoAllocScratchBytes)
     return set_error(SA_ERR_INVALID_ARG,
                      "pattern needs %zu bytes of plan data; the no-alloc entry point holds at most "
@@ -105,29 +108,23 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
 
   std::vector<int32_t> entries(cp.kb.size());
   for (size_t e = 0; e < cp.kb.size(); ++e) entries[e] = entry_pack(cp.kb[e], !cp.full[e]);
-  std::vector<int32_t> units(n_units);
-  std::iota(units.begin(), units.end(), 0);
-  auto cost = [&](int32_t u) {
-    const int t = u % T, h = (u / T) % H;
-    const int row = (cp.H_pat > 1 ? h : 0) * T + t;
-    return cp.row_ptr[row + 1] - cp.row_ptr[row];
-  };
-  std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
-    const int ca = cost(a), cb = cost(b);
-    if (ca != cb) return ca > cb;
-    return a % T != b % T ? a % T < b % T : a < b;
-  });
+  std::vector<int32_t> units;
+  order_units(cp, B, H, H_kv, &units);
 
   unsigned char* base = nullptr;
   rc = scratch_address(&base);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  int32_t* d_row = reinterpret_cast<int32_t*>(base);
-  int32_t* d_ent = reinterpret_cast<int32_t*>(base + b_row);
-  int32_t* d_units = reinterpret_cast<int32_t*>(base + b_row + b_ent);
-  int32_t* d_rtab = rnd ? reinterpret_cast<int32_t*>(base + b_row + b_ent + b_units) : nullptr;
-  cudaError_t e = cudaMemcpyAsync(d_row, cp.row_ptr.data(), cp.row_ptr.size() * 4,
-                                  cudaMemcpyHostToDevice, st);
+  int32_t* d_sched = reinterpret_cast<int32_t*>(base);
+  int32_t* d_row = reinterpret_cast<int32_t*>(base + b_sched);
+  int32_t* d_ent = reinterpret_cast<int32_t*>(base + b_sched + b_row);
+  int32_t* d_units = reinterpret_cast<int32_t*>(base + b_sched + b_row + b_ent);
+  int32_t* d_rtab =
+      rnd ? reinterpret_cast<int32_t*>(base + b_sched + b_row + b_ent + b_units) : nullptr;
+  cudaError_t e = cudaMemsetAsync(d_sched, 0, 2 * sizeof(int32_t), st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(d_row, cp.row_ptr.data(), cp.row_ptr.size() * 4, cudaMemcpyHostToDevice,
+                        st);
   if (e == cudaSuccess && !entries.empty())
     e = cudaMemcpyAsync(d_ent, entries.data(), entries.size() * 4, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess)
@@ -150,6 +147,7 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   p.row_ptr = d_row;
   p.entries = d_ent;
   p.units = d_units;
+  p.sched = d_sched;
   p.rtab = d_rtab;
   p.thresholds = pat->thresholds;
   p.n_units = int(n_units);

@@ -18,8 +18,10 @@
 //               mask of partial blocks, row max, tile max and gate, online
 //               softmax statistics (m, l) in fp32, P (bf16) written back over
 //               S in TMEM, lazy rescale of O, epilogue O / l.
-// Work units (b, h, tile) are taken in a longest-first order computed on the
-// host; CTA c takes units c, c + grid, c + 2*grid, ...
+// Work units (b, h, tile) come from a launch-wide queue: the host orders them
+// longest-first in coarse cost buckets (tile-major inside a bucket for K/V
+// locality in L2) and each CTA's producer claims the next one with an atomic
+// counter when it has room, so CTAs that get cheap units take more of them.
 //
 // TMEM columns: S buffer 0 at [0, 64), S buffer 1 at [64, 128), O at
 // [128, 128 + d).  P of a block overwrites the first 32 columns of its S
@@ -38,11 +40,15 @@ constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
 constexpr int kTmemO = 128;
 constexpr uint32_t kSoftmaxBar = 1;    // named barrier of the softmax warpgroup
+constexpr uint32_t kSoftmaxWarps = 4;
 constexpr float kRescaleLog2 = 8.0f;   // lazy rescale: keep a stale max up to 2^8
+constexpr uint32_t kUnitRing = 4;       // depth of the work-unit ring
+// consumers of a ring slot: the MMA thread and one lane of each softmax warp
+constexpr uint32_t kUnitConsumers = 1 + 4;
 
 // where-codes recorded with SA_ERR_TIMEOUT
 enum { W_PROD_Q = 1, W_PROD_K, W_MMA_Q, W_MMA_SFREE, W_MMA_K, W_MMA_VEMPTY, W_MMA_DEC,
-       W_MMA_P, W_MMA_VFULL, W_SM_S, W_SM_O, W_SM_EPI };
+       W_MMA_P, W_MMA_VFULL, W_SM_S, W_SM_O, W_SM_EPI, W_PROD_UNIT, W_MMA_UNIT, W_SM_UNIT };
 
 template <int D>
 struct Cfg {
@@ -69,10 +75,12 @@ struct Bars {
   uint64_t s_full[2], s_free[2], p_ready[2], dec[2];
   uint64_t o_done[2];
   uint64_t drain;
+  uint64_t u_full[4], u_empty[4];   // work-unit ring (producer -> MMA + softmax)
   uint32_t tmem_base;
   int abort;
   uint32_t flags[2];   // per S buffer: 1 = block kept, 0 = skipped
   float red[2][4];     // per S buffer: warp maxima for the tile maximum
+  int unit_slot[4];    // unit index, or -1 once the queue is exhausted
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block too large");
 
@@ -94,6 +102,43 @@ __device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
   return u;
 }
 
+// Work queue.  The producer thread claims unit indices from the launch-wide
+// counter p.sched[0] (atomicAdd, longest-first order) and publishes each in a
+// shared-memory ring; the MMA thread and the softmax warps take them from the
+// ring in the same order.  -1 marks the end of the queue.
+__device__ __forceinline__ bool publish_unit(const PrefillParams& p, Bars* bars, uint32_t n,
+                                             int* ui) {
+  const uint32_t slot = n % kUnitRing;
+  if (!wait_bounded(smem_u32(&bars->u_empty[slot]), ((n / kUnitRing) & 1) ^ 1, &bars->abort,
+                    p.err, W_PROD_UNIT))
+    return false;
+  int v = atomicAdd(p.sched, 1);
+  if (v >= p.n_units) v = -1;
+  reinterpret_cast<volatile int*>(bars->unit_slot)[slot] = v;
+  mbar_arrive(smem_u32(&bars->u_full[slot]));
+  *ui = v;
+  return true;
+}
+
+// Consumer side: one thread (MMA) or every lane of a softmax warp calls it;
+// the slot is released once per caller group (the warp's lane 0 after the
+// whole warp has read it).
+__device__ __forceinline__ bool take_unit(const PrefillParams& p, Bars* bars, uint32_t n, int* ui,
+                                          int where, bool whole_warp) {
+  const uint32_t slot = n % kUnitRing;
+  if (!wait_bounded(smem_u32(&bars->u_full[slot]), (n / kUnitRing) & 1, &bars->abort, p.err,
+                    where))
+    return false;
+  *ui = reinterpret_cast<volatile int*>(bars->unit_slot)[slot];
+  if (whole_warp) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&bars->u_empty[slot]));
+  } else {
+    mbar_arrive(smem_u32(&bars->u_empty[slot]));
+  }
+  return true;
+}
+
 // ------------------------------------------------------------ producer --
 template <int D>
 __device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars) {
@@ -102,7 +147,10 @@ __device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars)
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
   uint32_t qc = 0, kc = 0;
-  for (int ui = blockIdx.x; ui < p.n_units; ui += gridDim.x) {
+  for (uint32_t n = 0;; ++n) {
+    int ui;
+    if (!publish_unit(p, bars, n, &ui)) goto drain;
+    if (ui < 0) break;
     const Unit u = get_unit(p, ui);
     if (u.n == 0) continue;
     if (!wait_bounded(smem_u32(&bars->q_empty), (qc & 1) ^ 1, abort_flag, p.err, W_PROD_Q))
@@ -150,10 +198,19 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
   uint32_t qc = 0, kc = 0, g = 0, vc = 0, pvc = 0;
   bool ok = true;
 
-  for (int ui = blockIdx.x; ui < p.n_units && ok; ui += gridDim.x) {
+  for (uint32_t n = 0; ok; ++n) {
+    int ui;
+    if (!take_unit(p, bars, n, &ui, W_MMA_UNIT, false)) {
+      ok = false;
+      break;
+    }
+    if (ui < 0) break;
     const Unit u = get_unit(p, ui);
     if (u.n == 0) continue;
-    if (!wait_bounded(smem_u32(&bars->q_full), qc & 1, abort_flag, p.err, W_MMA_Q)) break;
+    if (!wait_bounded(smem_u32(&bars->q_full), qc & 1, abort_flag, p.err, W_MMA_Q)) {
+      ok = false;
+      break;
+    }
     ++qc;
     tc_fence_after();
     const uint32_t g0 = g;
@@ -275,33 +332,127 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Masks the logits of a partial block: x[c] = -inf for keys j = kb*64 + c
-// outside G_i (same predicate as the pattern compiler, evaluated per pair).
-__device__ __forceinline__ void mask_partial(const PrefillParams& p, int h, int i, int kb,
-                                             float (&x)[64]) {
+// Bits [lo, hi) of a 64-bit mask, with lo and hi clamped to [0, 64].
+__device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 64);
+  if (hi <= lo) return 0ull;
+  const uint64_t upto_hi = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
+  return upto_hi & ~((1ull << lo) - 1ull);
+}
+
+// Visible keys of row i inside block kb, as a 64-bit mask (bit c = key
+// kb*64 + c).  Every primitive is one index range per row (random blocks cover
+// whole 64-key blocks), so the union is built from ranges; the causal cap and
+// the sequence end are applied last.  Same predicate as the pattern compiler.
+__device__ __forceinline__ uint64_t visible_bits(const PrefillParams& p, int h, int i, int kb) {
+  if (i >= p.N) return 0ull;
   const int j0 = kb * kTileK;
-  const bool row_ok = i < p.N;
   const bool any_prim = p.window > 0 || p.n_global > 0 || p.block_local > 0 || p.n_random > 0;
-  bool rnd = false;
-  if (p.n_random > 0 && row_ok) {
-    const int nrb = (p.N + p.random_block - 1) / p.random_block;
-    const int32_t* row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
-    const int kr = j0 / p.random_block;
-    for (int r = 0; r < p.n_random; ++r) rnd |= __ldg(row + r) == kr;
+  uint64_t m = 0ull;
+  if (!any_prim || i < p.n_global) {
+    m = ~0ull;
+  } else {
+    if (p.n_global > 0) m |= range_bits(0, p.n_global - j0);
+    if (p.window > 0) {
+      if (p.causal) m |= range_bits(i - p.window + 1 - j0, i + 1 - j0);
+      else m |= range_bits(i - p.window / 2 - j0, i + p.window / 2 + 1 - j0);
+    }
+    if (p.block_local > 0) {
+      const int lo = (i / p.block_local) * p.block_local;
+      m |= range_bits(lo - j0, lo + p.block_local - j0);
+    }
+    if (p.n_random > 0) {
+      const int nrb = (p.N + p.random_block - 1) / p.random_block;
+      const int32_t* row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
+      const int kr = j0 / p.random_block;
+      bool rnd = false;
+      for (int r = 0; r < p.n_random; ++r) rnd |= __ldg(row + r) == kr;
+      if (rnd) m = ~0ull;
+    }
   }
-  const bool glob_row = i < p.n_global;
-  const int bl_lo = p.block_local > 0 ? (i / p.block_local) * p.block_local : 0;
-  const int bl_hi = p.block_local > 0 ? bl_lo + p.block_local : 0;
-  const int half_w = p.window / 2;
+  if (p.causal) m &= range_bits(0, i + 1 - j0);
+  m &= range_bits(0, p.N - j0);
+  return m;
+}
+
+// x[c] = -inf where bit c of the visibility mask is clear.
+__device__ __forceinline__ void apply_mask(uint64_t m, float (&x)[64]) {
+  const uint32_t lo = static_cast<uint32_t>(m), hi = static_cast<uint32_t>(m >> 32);
 #pragma unroll
-  for (int c = 0; c < 64; ++c) {
-    const int j = j0 + c;
-    bool v = !any_prim || glob_row || rnd || j < p.n_global;
-    if (p.window > 0) v |= p.causal ? (j > i - p.window) : (abs(i - j) <= half_w);
-    v |= (j >= bl_lo && j < bl_hi);
-    v = v && row_ok && j < p.N && (!p.causal || j <= i);
-    if (!v) x[c] = -INFINITY;
+  for (int c = 0; c < 32; ++c) {
+    if (!((lo >> c) & 1u)) x[c] = -INFINITY;
+    if (!((hi >> c) & 1u)) x[32 + c] = -INFINITY;
   }
+}
+
+// ---- softmax arithmetic on 64 logits per thread ----
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Row maximum as a tree of 3-input maxima (depth 4 instead of a 63-long chain).
+__device__ __forceinline__ float row_max64(const float (&x)[64]) {
+  float a[22];
+#pragma unroll
+  for (int k = 0; k < 21; ++k) a[k] = max3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+  a[21] = x[63];
+  float b[8];
+#pragma unroll
+  for (int k = 0; k < 7; ++k) b[k] = max3(a[3 * k], a[3 * k + 1], a[3 * k + 2]);
+  b[7] = a[21];
+  return max3(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
+}
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x for a pair, on the FMA pipe: x = n + f with n = floor(x) obtained by
+// adding 1.5*2^23 with round-down (the integer lands in the low mantissa
+// bits), f in [0, 1); 2^f by a degree-3 polynomial fitted by the Remez
+// exchange for minimum relative error on [0, 1] (max 7.5e-5, see
+// gen_exp2_poly.py); 2^n applied by adding n to the exponent field.  Inputs
+// below -125 (including -inf) give exactly 0.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  const float c0 = x0 < -125.f ? -125.f : x0;
+  const float c1 = x1 < -125.f ? -125.f : x1;
+  const float t0 = __fadd_rd(c0, kShift), t1 = __fadd_rd(c1, kShift);
+  const uint64_t t = f2_pack(t0, t1);
+  const uint64_t n = f2_sub(t, f2_pack(kShift, kShift));            // floor(x), exact
+  const uint64_t f = f2_sub(f2_pack(c0, c1), n);                     // in [0, 1)
+  uint64_t q = f2_fma(f2_pack(7.802452264e-02f, 7.802452264e-02f), f,
+                      f2_pack(2.260671554e-01f, 2.260671554e-01f));
+  q = f2_fma(q, f, f2_pack(6.958335405e-01f, 6.958335405e-01f));
+  q = f2_fma(q, f, f2_pack(9.999252186e-01f, 9.999252186e-01f));
+  float q0, q1;
+  f2_unpack(q, q0, q1);
+  const int n0 = __float_as_int(t0) - 0x4B400000, n1 = __float_as_int(t1) - 0x4B400000;
+  y0 = x0 < -125.f ? 0.f : __int_as_float(__float_as_int(q0) + (n0 << 23));
+  y1 = x1 < -125.f ? 0.f : __int_as_float(__float_as_int(q1) + (n1 << 23));
 }
 
 template <int D>
@@ -315,7 +466,10 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
   const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
   uint32_t g = 0, pv_total = 0;
 
-  for (int ui = blockIdx.x; ui < p.n_units; ui += gridDim.x) {
+  for (uint32_t n = 0;; ++n) {
+    int ui;
+    if (!take_unit(p, bars, n, &ui, W_SM_UNIT, true)) return;
+    if (ui < 0) break;
     const Unit u = get_unit(p, ui);
     const int i = u.t * kTileQ + row;
     const bool row_ok = i < p.N;
@@ -324,12 +478,17 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
     const float tau = (p.gate && !p.stats_only) ? __ldg(p.thresholds + u.h) : 0.f;
     float m = -INFINITY, l = 0.f;
     uint32_t kept = 0;
+    // Block entries are read one block ahead so the load overlaps the S wait.
+    int e_next = u.n > 0 ? __ldg(p.entries + u.beg) : 0;
 
     for (int k = 0; k < u.n; ++k) {
       const uint32_t buf = g & 1;
-      const int e = __ldg(p.entries + u.beg + k);
+      const int e = e_next;
+      if (k + 1 < u.n) e_next = __ldg(p.entries + u.beg + k + 1);
       const int kb = e >> 1;
       const bool partial = e & 1;
+      uint64_t vis = ~0ull;
+      if (partial) vis = visible_bits(p, u.h, i, kb);
       if (!wait_bounded(smem_u32(&bars->s_full[buf]), (g >> 1) & 1, abort_flag, p.err, W_SM_S))
         return;
       tc_fence_after();
@@ -346,10 +505,8 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         }
       }
       tc_fence_before();
-      if (partial) mask_partial(p, u.h, i, kb, x);
-      float mx = x[0];
-#pragma unroll
-      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+      if (partial) apply_mask(vis, x);
+      const float mx = row_max64(x);
 
       bool keep = true;
       if (p.want_stats) {
@@ -375,7 +532,7 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         // Every thread has read S (wait::ld + fence before the barrier above).
         if (leader) {
           mbar_arrive(smem_u32(&bars->s_free[buf]));
-          mbar_arrive(smem_u32(&bars->p_ready[buf]));
+          mbar_arrive_cnt(smem_u32(&bars->p_ready[buf]), kSoftmaxWarps);
         }
         ++g;
         continue;
@@ -411,24 +568,39 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         }
       }
       const float mb = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
+      // p = 2^(s*scale*log2e - m): the argument in packed f32x2 FMAs; one pair
+      // in four through the FMA-pipe polynomial, the rest through MUFU, so the
+      // two pipes share the exponentials.
+      constexpr int kPolyEvery = 4;
+      const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+      const uint64_t nmb = f2_pack(-mb, -mb);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2(fmaf(x[2 * c], p.scale_log2, -mb));
-        const float p1 = ex2(fmaf(x[2 * c + 1], p.scale_log2, -mb));
-        rs += p0 + p1;
+        float a0, a1, p0, p1;
+        f2_unpack(f2_fma(f2_pack(x[2 * c], x[2 * c + 1]), sl2, nmb), a0, a1);
+        if ((c % kPolyEvery) == kPolyEvery - 1) {
+          exp2_poly_pair(a0, a1, p0, p1);
+        } else {
+          p0 = ex2(a0);
+          p1 = ex2(a1);
+        }
+        acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
         pk[c] = pack_bf16x2(p0, p1);
       }
-      l += rs;
+      {
+        float s0, s1;
+        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
+        l += s0 + s1;
+      }
       tmem_st32(tmem + lane_base + buf * 64, pk);
       tmem_wait_st();
       tc_fence_before();
-      named_bar_sync(kSoftmaxBar, 128);
-      if (leader) {
-        flags[buf] = 1u;
-        mbar_arrive(smem_u32(&bars->p_ready[buf]));
-      }
+      // Each warp signals its own 32 rows of P; the MMA warp waits for all four.
+      if (leader) flags[buf] = 1u;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[buf]));
       ++kept;
       ++pv_total;
       ++g;
@@ -492,11 +664,15 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bars->s_full[b]), 1);
       mbar_init(smem_u32(&bars->s_free[b]), 1);
-      mbar_init(smem_u32(&bars->p_ready[b]), 1);
+      mbar_init(smem_u32(&bars->p_ready[b]), kSoftmaxWarps);
       mbar_init(smem_u32(&bars->dec[b]), 1);
       mbar_init(smem_u32(&bars->o_done[b]), 1);
     }
     mbar_init(smem_u32(&bars->drain), 1);
+    for (uint32_t r = 0; r < kUnitRing; ++r) {
+      mbar_init(smem_u32(&bars->u_full[r]), 1);
+      mbar_init(smem_u32(&bars->u_empty[r]), kUnitConsumers);
+    }
     bars->abort = 0;
     bars->flags[0] = bars->flags[1] = 0;
     fence_mbar_init();
@@ -527,6 +703,15 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  // The last CTA to finish resets the work-queue counters for the next launch
+  // (every CTA has claimed past the end of the queue before it gets here).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1) == int(gridDim.x) - 1) {
+      atomicExch(p.sched, 0);
+      atomicExch(p.sched + 1, 0);
+    }
+  }
 }
 
 int g_num_sms[64] = {0};

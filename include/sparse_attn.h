@@ -135,7 +135,10 @@ void sparse_attn_plan_destroy(sa_plan_t *plan);   /* synchronises the device; NU
  *   block_stat_out: device float [B][H][T_q][n_kb]; for listed blocks the
  *            maximum scaled logit over the tile's visible pairs (unlisted
  *            entries are left untouched); or NULL.
- * The plan must not be destroyed while a launch that uses it may still run. */
+ * The plan must not be destroyed while a launch that uses it may still run,
+ * and launches that use one plan must not overlap on the GPU (issue them on
+ * one stream, or order them): the plan holds the launch's work-queue
+ * counters. */
 int sparse_attn_prefill_plan(const sa_plan_t *plan, const void *Q, const void *K,
                              const void *V, void *O, const float *thresholds,
                              float *lse_out, uint8_t *block_mask_out,
