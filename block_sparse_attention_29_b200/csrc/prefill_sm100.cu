@@ -10,22 +10,26 @@
 // below it the block's V tile is never loaded and its PV product never issued.
 //
 // One CTA = 6 warps, persistent, two CTAs per SM (each owns 256 TMEM columns):
-//   warp 0      TMA producer: Q tile once per work unit, K blocks in a ring.
-//   warp 1      TMEM owner and single-thread tcgen05 issuer: S = Q K^T into one
-//               of two TMEM S buffers, O += P V with P read from TMEM; it also
-//               issues the V tile loads, after the gate has kept the block.
+//   warp 0      TMA producer: lane 0 loads the Q tile once per work unit and
+//               the K blocks into a ring; lane 1 loads the V tiles of kept
+//               blocks (after the gate decision when the rule is on).
+//   warp 1      TMEM owner and single-thread tcgen05 issuer: S = Q K^T into
+//               TMEM, O += P V with P read from TMEM, as an event loop that
+//               issues whichever step is ready.
 //   warps 2..5  softmax warpgroup, one query row per thread (TMEM lane):
 //               mask of partial blocks, row max, tile max and gate, online
-//               softmax statistics (m, l) in fp32, P (bf16) written back over
-//               S in TMEM, lazy rescale of O, epilogue O / l.
+//               softmax statistics (m, l) in fp32, P (bf16) written to TMEM,
+//               lazy rescale of O, epilogue O / l.
 // Work units (b, h, tile) come from a launch-wide queue: the host orders them
 // longest-first in coarse cost buckets (tile-major inside a bucket for K/V
 // locality in L2) and each CTA's producer claims the next one with an atomic
 // counter when it has room, so CTAs that get cheap units take more of them.
 //
-// TMEM columns: S buffer 0 at [0, 64), S buffer 1 at [64, 128), O at
-// [128, 128 + d).  P of a block overwrites the first 32 columns of its S
-// buffer (bf16 pairs).
+// TMEM columns: S at [0, 64), P buffers at [64, 96) and [96, 128) (bf16
+// pairs), O at [128, 128 + d).  S has one buffer: the next block's QK^T is
+// issued as soon as the softmax warps have loaded the current S into
+// registers, so it overlaps their exponentials; P has two, so the PV of one
+// block and the P of the next do not wait for each other.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -38,17 +42,22 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
-constexpr int kTmemO = 128;
+constexpr int kTmemS = 0;     // S of the current block: 64 fp32 columns
+constexpr int kTmemP = 64;    // two P buffers of 32 columns (64 bf16 per row)
+constexpr int kTmemO = 128;   // O accumulator: d fp32 columns
 constexpr uint32_t kSoftmaxBar = 1;    // named barrier of the softmax warpgroup
 constexpr uint32_t kSoftmaxWarps = 4;
 constexpr float kRescaleLog2 = 8.0f;   // lazy rescale: keep a stale max up to 2^8
 constexpr uint32_t kUnitRing = 4;       // depth of the work-unit ring
-// consumers of a ring slot: the MMA thread and one lane of each softmax warp
-constexpr uint32_t kUnitConsumers = 1 + 4;
+// consumers of a ring slot: the MMA thread, the V loader and one lane of
+// each softmax warp
+constexpr uint32_t kUnitConsumers = 1 + 1 + 4;
+constexpr uint32_t kDecRing = 4;        // depth of the gate-decision ring
 
 // where-codes recorded with SA_ERR_TIMEOUT
 enum { W_PROD_Q = 1, W_PROD_K, W_MMA_Q, W_MMA_SFREE, W_MMA_K, W_MMA_VEMPTY, W_MMA_DEC,
-       W_MMA_P, W_MMA_VFULL, W_SM_S, W_SM_O, W_SM_EPI, W_PROD_UNIT, W_MMA_UNIT, W_SM_UNIT };
+       W_MMA_P, W_MMA_VFULL, W_SM_S, W_SM_O, W_SM_EPI, W_PROD_UNIT, W_MMA_UNIT, W_SM_UNIT,
+       W_SM_P, W_VL_UNIT, W_VL_DEC, W_VL_EMPTY, W_MMA_LOOP, W_SM_DEC };
 
 template <int D>
 struct Cfg {
@@ -72,15 +81,19 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[3], k_empty[3];
   uint64_t v_full[3], v_empty[3];
-  uint64_t s_full[2], s_free[2], p_ready[2], dec[2];
+  uint64_t s_full, s_free;              // the single S buffer: written / read out
+  uint64_t p_ready[2];                  // per block parity: P written (or block skipped)
+  uint64_t dec_full[4], dec_empty[4];   // gate decisions, softmax -> V loader
+  uint64_t p_free[2];                   // per P buffer: the PV that read it is done
   uint64_t o_done[2];
   uint64_t drain;
   uint64_t u_full[4], u_empty[4];   // work-unit ring (producer -> MMA + softmax)
   uint32_t tmem_base;
   int abort;
-  uint32_t flags[2];   // per S buffer: 1 = block kept, 0 = skipped
-  float red[2][4];     // per S buffer: warp maxima for the tile maximum
+  uint32_t flags[2];   // per block parity: 1 = block kept, 0 = skipped
+  float red[2][4];     // per block parity: warp maxima for the tile maximum
   int unit_slot[4];    // unit index, or -1 once the queue is exhausted
+  uint32_t dec_val[4]; // decision ring: 1 = keep, 0 = skip
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block too large");
 
@@ -184,7 +197,60 @@ drain:
   }
 }
 
+// ------------------------------------------------------------- V loader --
+// Producer warp, lane 1: loads the V tile of every kept block, in block order,
+// as soon as a V stage is free.  With the rule on it takes each block's gate
+// decision from the decision ring first (skipped blocks load nothing).
+template <int D>
+__device__ void vloader_role(const PrefillParams& p, uint8_t* smem, Bars* bars) {
+  using C = Cfg<D>;
+  volatile int* abort_flag = &bars->abort;
+  const uint32_t sV = smem_u32(smem + C::OFF_V);
+  uint32_t vc = 0, g = 0;
+  for (uint32_t n = 0;; ++n) {
+    int ui;
+    if (!take_unit(p, bars, n, &ui, W_VL_UNIT, false)) goto drain;
+    if (ui < 0) break;
+    const Unit u = get_unit(p, ui);
+    for (int k = 0; k < u.n; ++k, ++g) {
+      bool keep = true;
+      if (p.gate) {
+        const uint32_t slot = g % kDecRing;
+        if (!wait_bounded(smem_u32(&bars->dec_full[slot]), (g / kDecRing) & 1, abort_flag, p.err,
+                          W_VL_DEC))
+          goto drain;
+        keep = reinterpret_cast<volatile uint32_t*>(bars->dec_val)[slot] != 0;
+        mbar_arrive(smem_u32(&bars->dec_empty[slot]));
+      }
+      if (!keep) continue;
+      const int kb = __ldg(p.entries + u.beg + k) >> 1;
+      const uint32_t vs = vc % C::VS;
+      if (!wait_bounded(smem_u32(&bars->v_empty[vs]), ((vc / C::VS) & 1) ^ 1, abort_flag, p.err,
+                        W_VL_EMPTY))
+        goto drain;
+      const uint32_t dst = sV + vs * C::KV_BYTES;
+      mbar_expect_tx(smem_u32(&bars->v_full[vs]), C::KV_BYTES);
+      for (int c = 0; c < C::CH; ++c)
+        tma_load_3d(dst + c * (kTileK * 128), &p.tm_v, smem_u32(&bars->v_full[vs]), c * 64,
+                    kb * kTileK, u.b * p.Hkv + u.hkv);
+      ++vc;
+    }
+  }
+  return;
+drain:
+  for (uint32_t s = 0; s < C::VS && s < vc; ++s) {
+    const uint32_t last = vc - 1 - ((vc - 1 - s) % C::VS);
+    wait_drain(smem_u32(&bars->v_full[s]), (last / C::VS) & 1);
+  }
+}
+
 // ----------------------------------------------------------- MMA issuer --
+// One thread, an event loop per work unit that never blocks on one condition
+// while another step is ready.  Steps, each issued in block order:
+//   S  : S_k = Q K_k^T once the softmax has read S_{k-1} out of TMEM and K_k
+//        is in shared memory (and at most one block ahead of the P hand-off);
+//   P  : take block k's P hand-off (kept or skipped) from the softmax;
+//   PV : O += P_k V_k for a kept block once V_k has landed.
 template <int D>
 __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint32_t tmem) {
   using C = Cfg<D>;
@@ -195,7 +261,7 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
   const uint32_t sV = smem_u32(smem + C::OFF_V);
   constexpr uint32_t idesc_s = make_idesc_bf16(kTileQ, kTileK, 0);
   constexpr uint32_t idesc_o = make_idesc_bf16(kTileQ, D, 1);
-  uint32_t qc = 0, kc = 0, g = 0, vc = 0, pvc = 0;
+  uint32_t qc = 0, kc = 0, g = 0, pvc = 0;
   bool ok = true;
 
   for (uint32_t n = 0; ok; ++n) {
@@ -214,100 +280,87 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
     ++qc;
     tc_fence_after();
     const uint32_t g0 = g;
-
-    // S_k = Q K_k^T into S buffer (g & 1).
-    auto issue_s = [&](int k) -> bool {
-      const uint32_t buf = g & 1;
-      if (!wait_bounded(smem_u32(&bars->s_free[buf]), ((g >> 1) & 1) ^ 1, abort_flag, p.err,
-                        W_MMA_SFREE))
-        return false;
-      const uint32_t st = kc % C::KS;
-      if (!wait_bounded(smem_u32(&bars->k_full[st]), (kc / C::KS) & 1, abort_flag, p.err, W_MMA_K))
-        return false;
-      tc_fence_after();
-      const uint32_t kbase = sK + st * C::KV_BYTES;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * 0 + (kk & 3) * 32;
-        const uint64_t da = make_sdesc(sQ + (kk >> 2) * (kTileQ * 128) + off, 16, 1024);
-        const uint64_t db = make_sdesc(kbase + (kk >> 2) * (kTileK * 128) + off, 16, 1024);
-        umma_ss(tmem + buf * 64, da, db, idesc_s, kk > 0 ? 1u : 0u);
-      }
-      tc_commit(smem_u32(&bars->k_empty[st]));
-      tc_commit(smem_u32(&bars->s_full[buf]));
-      if (k == u.n - 1) tc_commit(smem_u32(&bars->q_empty));
-      ++kc;
-      ++g;
-      return true;
-    };
-    // TMA load of V block k into the next V stage.
-    auto issue_v = [&](int k) -> bool {
-      const int kb = __ldg(p.entries + u.beg + k) >> 1;
-      const uint32_t vs = vc % C::VS;
-      if (!wait_bounded(smem_u32(&bars->v_empty[vs]), ((vc / C::VS) & 1) ^ 1, abort_flag, p.err,
-                        W_MMA_VEMPTY))
-        return false;
-      const uint32_t dst = sV + vs * C::KV_BYTES;
-      mbar_expect_tx(smem_u32(&bars->v_full[vs]), C::KV_BYTES);
-      for (int c = 0; c < C::CH; ++c)
-        tma_load_3d(dst + c * (kTileK * 128), &p.tm_v, smem_u32(&bars->v_full[vs]), c * 64,
-                    kb * kTileK, u.b * p.Hkv + u.hkv);
-      ++vc;
-      return true;
-    };
-    // Gate decision of block k (global block index g0 + k).
-    auto decision = [&](int k, bool* keep) -> bool {
-      const uint32_t gk = g0 + k;
-      if (!wait_bounded(smem_u32(&bars->dec[gk & 1]), (gk >> 1) & 1, abort_flag, p.err, W_MMA_DEC))
-        return false;
-      *keep = flags[gk & 1] != 0;
-      return true;
-    };
-
-    ok = issue_s(0) && (p.gate || issue_v(0));
-    if (ok && u.n > 1) ok = issue_s(1) && (p.gate || issue_v(1));
-    if (ok && p.gate) {
-      bool keep;
-      ok = decision(0, &keep) && (!keep || issue_v(0));
-    }
+    int ns = 0, nr = 0, npv = 0;   // S issued, P hand-offs taken, PVs handled
+    uint32_t keep_bits = 0;        // keep flags of blocks nr-? .. nr-1 (bit = block % 32)
     bool first_pv = true;
-    for (int k = 0; k < u.n && ok; ++k) {
-      const uint32_t gk = g0 + k, buf = gk & 1;
-      if (!wait_bounded(smem_u32(&bars->p_ready[buf]), (gk >> 1) & 1, abort_flag, p.err, W_MMA_P)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (flags[buf]) {
-        const uint32_t vs = pvc % C::VS;
-        if (!wait_bounded(smem_u32(&bars->v_full[vs]), (pvc / C::VS) & 1, abort_flag, p.err,
-                          W_MMA_VFULL)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t vbase = sV + vs * C::KV_BYTES;
+    uint64_t t_last = 0;
+    uint32_t idle = 0;
+    while (npv < u.n) {
+      bool progress = false;
+      // S for block ns.
+      if (ns < u.n && ns <= nr + 1) {
+        const uint32_t st = kc % C::KS;
+        if (mbar_try_wait(smem_u32(&bars->s_free), ((g0 + ns) & 1) ^ 1) &&
+            mbar_try_wait(smem_u32(&bars->k_full[st]), (kc / C::KS) & 1)) {
+          tc_fence_after();
+          const uint32_t kbase = sK + st * C::KV_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < kTileK / 16; ++kk) {
-          const uint64_t db = make_sdesc(vbase + kk * (16 * 128), kTileK * 128, 1024);
-          umma_ts(tmem + kTmemO, tmem + buf * 64 + kk * 8, db, idesc_o,
-                  (first_pv && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t da = make_sdesc(sQ + (kk >> 2) * (kTileQ * 128) + off, 16, 1024);
+            const uint64_t db = make_sdesc(kbase + (kk >> 2) * (kTileK * 128) + off, 16, 1024);
+            umma_ss(tmem + kTmemS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&bars->k_empty[st]));
+          tc_commit(smem_u32(&bars->s_full));
+          if (ns == u.n - 1) tc_commit(smem_u32(&bars->q_empty));
+          ++kc;
+          ++g;
+          ++ns;
+          progress = true;
         }
-        tc_commit(smem_u32(&bars->v_empty[vs]));
-        tc_commit(smem_u32(&bars->s_free[buf]));
-        tc_commit(smem_u32(&bars->o_done[pvc & 1]));
-        ++pvc;
-        first_pv = false;
       }
-      if (p.gate && k + 1 < u.n) {
-        bool keep;
-        if (!decision(k + 1, &keep) || (keep && !issue_v(k + 1))) {
+      // P hand-off of block nr.
+      if (nr < ns) {
+        const uint32_t gk = g0 + nr, fb = gk & 1;
+        if (mbar_try_wait(smem_u32(&bars->p_ready[fb]), (gk >> 1) & 1)) {
+          tc_fence_after();
+          if (flags[fb]) keep_bits |= 1u << (nr & 31);
+          else keep_bits &= ~(1u << (nr & 31));
+          ++nr;
+          progress = true;
+        }
+      }
+      // PV of block npv.
+      if (npv < nr) {
+        if (!((keep_bits >> (npv & 31)) & 1u)) {
+          ++npv;
+          progress = true;
+        } else {
+          const uint32_t vs = pvc % C::VS;
+          if (mbar_try_wait(smem_u32(&bars->v_full[vs]), (pvc / C::VS) & 1)) {
+            tc_fence_after();
+            const uint32_t vbase = sV + vs * C::KV_BYTES;
+            const uint32_t pcol = kTmemP + (pvc & 1) * 32;
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              const uint64_t db = make_sdesc(vbase + kk * (16 * 128), kTileK * 128, 1024);
+              umma_ts(tmem + kTmemO, tmem + pcol + kk * 8, db, idesc_o,
+                      (first_pv && kk == 0) ? 0u : 1u);
+            }
+            tc_commit(smem_u32(&bars->v_empty[vs]));
+            tc_commit(smem_u32(&bars->p_free[pvc & 1]));
+            tc_commit(smem_u32(&bars->o_done[pvc & 1]));
+            ++pvc;
+            ++npv;
+            first_pv = false;
+            progress = true;
+          }
+        }
+      }
+      if (progress) {
+        idle = 0;
+      } else if ((++idle & 255u) == 0) {
+        // Bounded: no step became ready for the whole wait budget -> abort.
+        if (*abort_flag) {
           ok = false;
           break;
         }
-      }
-      if (k + 2 < u.n) {
-        if (!issue_s(k + 2) || (!p.gate && !issue_v(k + 2))) {
+        const uint64_t now = globaltimer_ns();
+        if (idle == 256) t_last = now;
+        else if (now - t_last > kWaitBudgetNs) {
+          record_device_error(p.err, SA_ERR_TIMEOUT, W_MMA_LOOP);
+          *abort_flag = 1;
           ok = false;
           break;
         }
@@ -315,13 +368,9 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
     }
   }
   if (!ok) {
-    // Let every MMA already issued finish, and V loads already issued land.
+    // Let every MMA already issued finish before TMEM and shared memory go away.
     tc_commit(smem_u32(&bars->drain));
     wait_drain(smem_u32(&bars->drain), 0);
-    for (uint32_t s = 0; s < C::VS && s < vc; ++s) {
-      const uint32_t last = vc - 1 - ((vc - 1 - s) % C::VS);
-      wait_drain(smem_u32(&bars->v_full[s]), (last / C::VS) & 1);
-    }
   }
 }
 
@@ -341,11 +390,36 @@ __device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
   return upto_hi & ~((1ull << lo) - 1ull);
 }
 
+// A row's random key blocks, read once per work unit (the row's random-block
+// row does not change inside a unit): up to kRowRandom held in registers,
+// longer lists read from global memory.
+constexpr int kRowRandom = 3;
+struct RowRandom {
+  int n;
+  int v[kRowRandom];
+  const int32_t* row;
+};
+
+__device__ __forceinline__ RowRandom load_row_random(const PrefillParams& p, int h, int i) {
+  RowRandom rr;
+  rr.n = 0;
+  rr.row = nullptr;
+  if (p.n_random > 0 && i < p.N) {
+    const int nrb = (p.N + p.random_block - 1) / p.random_block;
+    rr.row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
+    rr.n = p.n_random;
+#pragma unroll
+    for (int r = 0; r < kRowRandom; ++r) rr.v[r] = r < rr.n ? __ldg(rr.row + r) : -1;
+  }
+  return rr;
+}
+
 // Visible keys of row i inside block kb, as a 64-bit mask (bit c = key
 // kb*64 + c).  Every primitive is one index range per row (random blocks cover
 // whole 64-key blocks), so the union is built from ranges; the causal cap and
 // the sequence end are applied last.  Same predicate as the pattern compiler.
-__device__ __forceinline__ uint64_t visible_bits(const PrefillParams& p, int h, int i, int kb) {
+__device__ __forceinline__ uint64_t visible_bits(const PrefillParams& p, const RowRandom& rr,
+                                                 int i, int kb) {
   if (i >= p.N) return 0ull;
   const int j0 = kb * kTileK;
   const bool any_prim = p.window > 0 || p.n_global > 0 || p.block_local > 0 || p.n_random > 0;
@@ -362,12 +436,12 @@ __device__ __forceinline__ uint64_t visible_bits(const PrefillParams& p, int h, 
       const int lo = (i / p.block_local) * p.block_local;
       m |= range_bits(lo - j0, lo + p.block_local - j0);
     }
-    if (p.n_random > 0) {
-      const int nrb = (p.N + p.random_block - 1) / p.random_block;
-      const int32_t* row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
+    if (rr.n > 0) {
       const int kr = j0 / p.random_block;
       bool rnd = false;
-      for (int r = 0; r < p.n_random; ++r) rnd |= __ldg(row + r) == kr;
+#pragma unroll
+      for (int r = 0; r < kRowRandom; ++r) rnd |= rr.v[r] == kr;
+      for (int r = kRowRandom; r < rr.n; ++r) rnd |= __ldg(rr.row + r) == kr;
       if (rnd) m = ~0ull;
     }
   }
@@ -480,23 +554,23 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
     uint32_t kept = 0;
     // Block entries are read one block ahead so the load overlaps the S wait.
     int e_next = u.n > 0 ? __ldg(p.entries + u.beg) : 0;
+    const RowRandom rr = load_row_random(p, u.h, i);
 
     for (int k = 0; k < u.n; ++k) {
-      const uint32_t buf = g & 1;
+      const uint32_t fb = g & 1;   // per-block-parity flag / decision slot
       const int e = e_next;
       if (k + 1 < u.n) e_next = __ldg(p.entries + u.beg + k + 1);
       const int kb = e >> 1;
       const bool partial = e & 1;
       uint64_t vis = ~0ull;
-      if (partial) vis = visible_bits(p, u.h, i, kb);
-      if (!wait_bounded(smem_u32(&bars->s_full[buf]), (g >> 1) & 1, abort_flag, p.err, W_SM_S))
-        return;
+      if (partial) vis = visible_bits(p, rr, i, kb);
+      if (!wait_bounded(smem_u32(&bars->s_full), g & 1, abort_flag, p.err, W_SM_S)) return;
       tc_fence_after();
       float x[64];
       {
         uint32_t r0[32], r1[32];
-        tmem_ld32(tmem + lane_base + buf * 64, r0);
-        tmem_ld32(tmem + lane_base + buf * 64 + 32, r1);
+        tmem_ld32(tmem + lane_base + kTmemS, r0);
+        tmem_ld32(tmem + lane_base + kTmemS + 32, r1);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -504,36 +578,41 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
           x[32 + c] = __uint_as_float(r1[c]);
         }
       }
+      // S is in registers: release the S columns for the next block's QK^T.
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
       if (partial) apply_mask(vis, x);
       const float mx = row_max64(x);
 
       bool keep = true;
       if (p.want_stats) {
         const float wm = warp_max(mx);
-        if (lane == 0) bars->red[buf][q4] = wm;
+        if (lane == 0) bars->red[fb][q4] = wm;
         named_bar_sync(kSoftmaxBar, 128);
-        const float tmax = fmaxf(fmaxf(bars->red[buf][0], bars->red[buf][1]),
-                                 fmaxf(bars->red[buf][2], bars->red[buf][3]));
+        const float tmax = fmaxf(fmaxf(bars->red[fb][0], bars->red[fb][1]),
+                                 fmaxf(bars->red[fb][2], bars->red[fb][3]));
         const float stat = tmax * p.scale;
         if (p.gate) keep = !p.stats_only && (partial || !(stat < tau));
         if (leader) {
           if (p.stat_out) p.stat_out[tile_base + kb] = stat;
           if (p.mask_out) p.mask_out[tile_base + kb] = keep || p.stats_only ? 1 : 2;
           if (p.gate) {
-            flags[buf] = keep ? 1u : 0u;
-            mbar_arrive(smem_u32(&bars->dec[buf]));
+            flags[fb] = keep ? 1u : 0u;
+            const uint32_t slot = g % kDecRing;
+            // The V loader frees a slot as soon as it reads it; bounded wait.
+            if (wait_bounded(smem_u32(&bars->dec_empty[slot]), ((g / kDecRing) & 1) ^ 1, abort_flag,
+                             p.err, W_SM_DEC)) {
+              reinterpret_cast<volatile uint32_t*>(bars->dec_val)[slot] = keep ? 1u : 0u;
+              mbar_arrive(smem_u32(&bars->dec_full[slot]));
+            }
           }
         }
       } else if (leader && p.mask_out) {
         p.mask_out[tile_base + kb] = 1;
       }
       if (!keep) {
-        // Every thread has read S (wait::ld + fence before the barrier above).
-        if (leader) {
-          mbar_arrive(smem_u32(&bars->s_free[buf]));
-          mbar_arrive_cnt(smem_u32(&bars->p_ready[buf]), kSoftmaxWarps);
-        }
+        if (leader) mbar_arrive_cnt(smem_u32(&bars->p_ready[fb]), kSoftmaxWarps);
         ++g;
         continue;
       }
@@ -548,9 +627,14 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         l *= alpha;
         m = m_new;
       }
+      // This block's P goes to P buffer (pv_total & 1), free once the PV two
+      // before it has completed; after this wait at most one PV is in flight.
+      const uint32_t pb = pv_total & 1;
+      if (!wait_bounded(smem_u32(&bars->p_free[pb]), ((pv_total >> 1) & 1) ^ 1, abort_flag, p.err,
+                        W_SM_P))
+        return;
       if (kept > 0 && __any_sync(0xffffffffu, need)) {
-        // O += P V of the previous kept block must be complete before O is
-        // rescaled; at most one PV is in flight here.
+        // O += P V of the previous kept block must be complete before O is rescaled.
         const uint32_t last = pv_total - 1;
         if (!wait_bounded(smem_u32(&bars->o_done[last & 1]), (last >> 1) & 1, abort_flag, p.err,
                           W_SM_O))
@@ -594,13 +678,13 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
         l += s0 + s1;
       }
-      tmem_st32(tmem + lane_base + buf * 64, pk);
+      tmem_st32(tmem + lane_base + kTmemP + pb * 32, pk);
       tmem_wait_st();
       tc_fence_before();
       // Each warp signals its own 32 rows of P; the MMA warp waits for all four.
-      if (leader) flags[buf] = 1u;
+      if (leader) flags[fb] = 1u;
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[buf]));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[fb]));
       ++kept;
       ++pv_total;
       ++g;
@@ -661,14 +745,18 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
       mbar_init(smem_u32(&bars->v_full[s]), 1);
       mbar_init(smem_u32(&bars->v_empty[s]), 1);
     }
+    mbar_init(smem_u32(&bars->s_full), 1);
+    mbar_init(smem_u32(&bars->s_free), kSoftmaxWarps);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&bars->s_full[b]), 1);
-      mbar_init(smem_u32(&bars->s_free[b]), 1);
+      mbar_init(smem_u32(&bars->p_free[b]), 1);
       mbar_init(smem_u32(&bars->p_ready[b]), kSoftmaxWarps);
-      mbar_init(smem_u32(&bars->dec[b]), 1);
       mbar_init(smem_u32(&bars->o_done[b]), 1);
     }
     mbar_init(smem_u32(&bars->drain), 1);
+    for (uint32_t r = 0; r < kDecRing; ++r) {
+      mbar_init(smem_u32(&bars->dec_full[r]), 1);
+      mbar_init(smem_u32(&bars->dec_empty[r]), 1);
+    }
     for (uint32_t r = 0; r < kUnitRing; ++r) {
       mbar_init(smem_u32(&bars->u_full[r]), 1);
       mbar_init(smem_u32(&bars->u_empty[r]), kUnitConsumers);
@@ -693,6 +781,7 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
 
   if (warp == 0) {
     if (lane == 0) producer_role<D>(p, smem, bars);
+    else if (lane == 1) vloader_role<D>(p, smem, bars);
   } else if (warp == 1) {
     if (lane == 0) mma_role<D>(p, smem, bars, tmem);
   } else {
