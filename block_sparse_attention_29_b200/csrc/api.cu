@@ -317,7 +317,7 @@ int sparse_attn_plan_create(const sa_pattern_t* pat, int B, int H, int H_kv, int
 
   plan->n_units = B * cp.T * H;
   std::vector<int32_t> units;
-  order_units(cp, B, H, H_kv, &units);
+  order_units(cp, B, H, H_kv, int64_t(B) * H_kv * N * d * 2 * 2, &units);
 
   rc = upload(&plan->d_row_ptr, cp.row_ptr.data(), cp.row_ptr.size());
   if (!rc) rc = upload(&plan->d_entries, entries.data(), entries.size());

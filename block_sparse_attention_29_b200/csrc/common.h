@@ -101,8 +101,12 @@ int compile_pattern(const sa_pattern_t* pat, int H, int N, int tile_q, int tile_
                     CompiledPattern* out);
 // Validates the descriptor fields that do not depend on the kernel.
 int validate_pattern(const sa_pattern_t* pat, int H, int N);
-// Work order of the B*H*T units (unit = (b*H + h)*T + t): longest first in
-// coarse cost buckets, tile-major with GQA siblings adjacent inside a bucket.
-void order_units(const CompiledPattern& cp, int B, int H, int H_kv, std::vector<int32_t>* units);
+// Work order of the B*H*T units (unit = (b*H + h)*T + t): units longer than
+// half a CTA's share first (longest first), the rest tile-major or
+// K/V-group-major (see kv_bytes), the query heads of a group adjacent.
+// kv_bytes: size of K plus V; above 64 MiB (half of L2) the order is
+// K/V-group-major, below tile-major.
+void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_bytes,
+                 std::vector<int32_t>* units);
 
 }  // namespace sa

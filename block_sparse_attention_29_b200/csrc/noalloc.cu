@@ -109,7 +109,7 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   std::vector<int32_t> entries(cp.kb.size());
   for (size_t e = 0; e < cp.kb.size(); ++e) entries[e] = entry_pack(cp.kb[e], !cp.full[e]);
   std::vector<int32_t> units;
-  order_units(cp, B, H, H_kv, &units);
+  order_units(cp, B, H, H_kv, int64_t(B) * H_kv * N * d * 2 * 2, &units);
 
   unsigned char* base = nullptr;
   rc = scratch_address(&base);

@@ -151,7 +151,8 @@ int compile_pattern(const sa_pattern_t* p, int H, int N, int tile_q, int tile_k,
   return SA_OK;
 }
 
-void order_units(const CompiledPattern& cp, int B, int H, int H_kv, std::vector<int32_t>* out) {
+void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_bytes,
+                 std::vector<int32_t>* out) {
   const int T = cp.T;
   const int64_t n = int64_t(B) * H * T;
   out->resize(size_t(n));
@@ -162,24 +163,34 @@ void order_units(const CompiledPattern& cp, int B, int H, int H_kv, std::vector<
     const int row = (cp.H_pat > 1 ? h : 0) * T + t;
     return cp.row_ptr[row + 1] - cp.row_ptr[row];
   };
-  int max_cost = 1;
-  for (int r = 0; r + 1 < int(cp.row_ptr.size()); ++r)
-    max_cost = std::max(max_cost, cp.row_ptr[r + 1] - cp.row_ptr[r]);
-  // Longest first at a coarse grain (16 cost buckets), so the expensive units
-  // start early; inside a bucket tile-major (later tiles first, the larger
-  // ones under a causal mask) with (b, kv head, head) innermost, so the units
-  // that read the same K/V blocks run close together in time.
-  auto bucket = [&](int32_t u) { return int64_t(16) * cost(u) / (int64_t(max_cost) + 1); };
+  int64_t total = 0;
+  for (int64_t u = 0; u < n; ++u) total += cost(int32_t(u));
+  // Units longer than half of one CTA's share of the work (2 CTAs per SM on
+  // a 148-SM part) would set the tail if they started late: they go first,
+  // longest first.  When all of K and V fit in half of L2 the rest are
+  // ordered tile-major (later tiles first, the larger ones under a causal
+  // mask); otherwise K/V-group-major -- all tiles of the query heads that
+  // share one K/V head run together, so that head's K and V stay in L2 while
+  // they are reused -- longest first inside a group.  The query heads of a
+  // group are adjacent either way.
+  const int64_t heavy = std::max<int64_t>(1, total / (2 * 296) / 2);
+  const bool group_major = kv_bytes > (int64_t(64) << 20);
   const int group = H / H_kv;
   std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
-    const int64_t ca = bucket(a), cb = bucket(b);
-    if (ca != cb) return ca > cb;
-    const int ta = a % T, tb = b % T;
-    if (ta != tb) return ta > tb;
+    const int ca = cost(a), cb = cost(b);
+    const bool ha_ = ca > heavy, hb_ = cb > heavy;
+    if (ha_ != hb_) return ha_;
+    if (ha_ && ca != cb) return ca > cb;
     const int bha = a / T, bhb = b / T;
     const int ba = bha / H, bb = bhb / H, ha = bha % H, hb = bhb % H;
+    if (!ha_ && group_major) {
+      if (ba != bb) return ba < bb;
+      if (ha / group != hb / group) return ha / group < hb / group;
+      if (ca != cb) return ca > cb;
+    }
+    const int ta = a % T, tb = b % T;
+    if (ta != tb) return ta > tb;
     if (ba != bb) return ba < bb;
-    if (ha / group != hb / group) return ha / group < hb / group;
     return ha < hb;
   });
 }

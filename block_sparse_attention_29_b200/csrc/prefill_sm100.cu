@@ -21,9 +21,10 @@
 //               softmax statistics (m, l) in fp32, P (bf16) written to TMEM,
 //               lazy rescale of O, epilogue O / l.
 // Work units (b, h, tile) come from a launch-wide queue: the host orders them
-// longest-first in coarse cost buckets (tile-major inside a bucket for K/V
-// locality in L2) and each CTA's producer claims the next one with an atomic
-// counter when it has room, so CTAs that get cheap units take more of them.
+// (very long units first; then tile-major when all of K/V fits in L2, else
+// K/V-group-major so a K/V head's blocks stay in L2 while its query heads use
+// them) and each CTA's producer claims the next one with an atomic counter
+// when it has room, so CTAs that get cheap units take more of them.
 //
 // TMEM columns: S at [0, 64), P buffers at [64, 96) and [96, 128) (bf16
 // pairs), O at [128, 128 + d).  S has one buffer: the next block's QK^T is
