@@ -138,6 +138,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
+# ------------------------------------------------------------ multi-rank --
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world: int, work_per_rank: float, seconds: float, scale: float) -> float:
+    """Whole-job throughput of `world` independent replicas that each did
+    `work_per_rank` units of work, timed by the slowest rank (max over ranks)."""
+    return world * work_per_rank / seconds / scale
+
+
 # ---------------------------------------------------------------- workloads --
 def prefill_accounting(w, info, kept_desc=None, skipped_pairs=0):
     """FLOPs of one prefill launch: computed-block (descriptor granularity),
@@ -360,10 +377,7 @@ def main():
     sa.check_device_error()
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sum(per_step)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, device)
     ms_per_step = total_ms / args.steps
 
     # end to end: the same call with host buffers, copies inside the timed region
@@ -378,23 +392,20 @@ def main():
         S["e2e_step"](stream)
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / args.steps
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device) / args.steps
     sa.check_device_error()
 
     peaks, peak_src = load_peaks()
     per_launch_s = ms_per_step / 1e3
     if S["unit"] == "TFLOP/s":
-        value = world * S["flops"] / per_launch_s / 1e12
-        e2e_value = world * S["flops"] / (e2e_ms / 1e3) / 1e12
+        value = aggregate_rate(world, S["flops"], per_launch_s, 1e12)
+        e2e_value = aggregate_rate(world, S["flops"], e2e_ms / 1e3, 1e12)
         achieved = S["flops"] / per_launch_s / 1e12
         peak = peaks["bf16_tflops"]
         roof_unit = "TFLOP/s"
     else:
-        value = world * S["algo_bytes"] / per_launch_s / 1e9
-        e2e_value = world * S["algo_bytes"] / (e2e_ms / 1e3) / 1e9
+        value = aggregate_rate(world, S["algo_bytes"], per_launch_s, 1e9)
+        e2e_value = aggregate_rate(world, S["algo_bytes"], e2e_ms / 1e3, 1e9)
         achieved = value / world
         peak = peaks["hbm_gbs"]
         roof_unit = "GB/s"
