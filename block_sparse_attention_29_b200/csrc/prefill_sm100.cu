@@ -499,36 +499,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-// 2^x for a pair, on the FMA pipe: x = n + f with n = floor(x) obtained by
-// adding 1.5*2^23 with round-down (the integer lands in the low mantissa
-// bits), f in [0, 1); 2^f by a degree-3 polynomial fitted by the Remez
-// exchange for minimum relative error on [0, 1] (max 7.5e-5, see
-// gen_exp2_poly.py); 2^n applied by adding n to the exponent field.  Inputs
-// below -125 (including -inf) give exactly 0.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
-  const float c0 = x0 < -125.f ? -125.f : x0;
-  const float c1 = x1 < -125.f ? -125.f : x1;
-  const float t0 = __fadd_rd(c0, kShift), t1 = __fadd_rd(c1, kShift);
-  const uint64_t t = f2_pack(t0, t1);
-  const uint64_t n = f2_sub(t, f2_pack(kShift, kShift));            // floor(x), exact
-  const uint64_t f = f2_sub(f2_pack(c0, c1), n);                     // in [0, 1)
-  uint64_t q = f2_fma(f2_pack(7.802452264e-02f, 7.802452264e-02f), f,
-                      f2_pack(2.260671554e-01f, 2.260671554e-01f));
-  q = f2_fma(q, f, f2_pack(6.958335405e-01f, 6.958335405e-01f));
-  q = f2_fma(q, f, f2_pack(9.999252186e-01f, 9.999252186e-01f));
-  float q0, q1;
-  f2_unpack(q, q0, q1);
-  const int n0 = __float_as_int(t0) - 0x4B400000, n1 = __float_as_int(t1) - 0x4B400000;
-  y0 = x0 < -125.f ? 0.f : __int_as_float(__float_as_int(q0) + (n0 << 23));
-  y1 = x1 < -125.f ? 0.f : __int_as_float(__float_as_int(q1) + (n1 << 23));
-}
 
 template <int D>
 __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, int warp,
@@ -653,10 +623,10 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         }
       }
       const float mb = (m == -INFINITY) ? 0.f : m;
-      // p = 2^(s*scale*log2e - m): the argument in packed f32x2 FMAs; one pair
-      // in four through the FMA-pipe polynomial, the rest through MUFU, so the
-      // two pipes share the exponentials.
-      constexpr int kPolyEvery = 4;
+      // p = 2^(s*scale*log2e - m): the argument and the row sum in packed
+      // f32x2 arithmetic, the exponentials on MUFU (ex2.approx).  Moving part
+      // of them to an FMA-pipe polynomial was measured slower: this loop is
+      // bound by instruction issue, not by the MUFU pipe.
       const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
       const uint64_t nmb = f2_pack(-mb, -mb);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -665,12 +635,8 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       for (int c = 0; c < 32; ++c) {
         float a0, a1, p0, p1;
         f2_unpack(f2_fma(f2_pack(x[2 * c], x[2 * c + 1]), sl2, nmb), a0, a1);
-        if ((c % kPolyEvery) == kPolyEvery - 1) {
-          exp2_poly_pair(a0, a1, p0, p1);
-        } else {
-          p0 = ex2(a0);
-          p1 = ex2(a1);
-        }
+        p0 = ex2(a0);
+        p1 = ex2(a1);
         acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
         pk[c] = pack_bf16x2(p0, p1);
       }
