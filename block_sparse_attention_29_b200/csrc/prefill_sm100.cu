@@ -376,10 +376,11 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
 }
 
 // --------------------------------------------------------------- softmax --
+// Maximum over the 32 lanes of a warp (one redux instruction on sm_100a).
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 
 // Bits [lo, hi) of a 64-bit mask, with lo and hi clamped to [0, 64].
@@ -535,6 +536,12 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       const bool partial = e & 1;
       uint64_t vis = ~0ull;
       if (partial) vis = visible_bits(p, rr, i, kb);
+      // The leader claims this block's decision-ring slot now, while S is
+      // still being computed (the V loader frees slots as it reads them).
+      bool slot_ok = true;
+      if (leader && p.gate)
+        slot_ok = wait_bounded(smem_u32(&bars->dec_empty[g % kDecRing]),
+                               ((g / kDecRing) & 1) ^ 1, abort_flag, p.err, W_SM_DEC);
       if (!wait_bounded(smem_u32(&bars->s_full), g & 1, abort_flag, p.err, W_SM_S)) return;
       tc_fence_after();
       float x[64];
@@ -570,10 +577,8 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
           if (p.mask_out) p.mask_out[tile_base + kb] = keep || p.stats_only ? 1 : 2;
           if (p.gate) {
             flags[fb] = keep ? 1u : 0u;
-            const uint32_t slot = g % kDecRing;
-            // The V loader frees a slot as soon as it reads it; bounded wait.
-            if (wait_bounded(smem_u32(&bars->dec_empty[slot]), ((g / kDecRing) & 1) ^ 1, abort_flag,
-                             p.err, W_SM_DEC)) {
+            if (slot_ok) {
+              const uint32_t slot = g % kDecRing;
               reinterpret_cast<volatile uint32_t*>(bars->dec_val)[slot] = keep ? 1u : 0u;
               mbar_arrive(smem_u32(&bars->dec_full[slot]));
             }
