@@ -78,6 +78,10 @@ struct Cfg {
   static constexpr int SMEM = (SMEM_USED > 80 * 1024 ? SMEM_USED : 80 * 1024) + 1024;
 };
 
+struct Unit {
+  int b, h, hkv, t, beg, n;
+};
+
 struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[3], k_empty[3];
@@ -93,14 +97,11 @@ struct Bars {
   int abort;
   uint32_t flags[2];   // per block parity: 1 = block kept, 0 = skipped
   float red[2][4];     // per block parity: warp maxima for the tile maximum
-  int unit_slot[4];    // unit index, or -1 once the queue is exhausted
+  Unit unit_slot[4];   // decoded work unit; n = -1 once the queue is exhausted
   uint32_t dec_val[4]; // decision ring: 1 = keep, 0 = skip
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block too large");
 
-struct Unit {
-  int b, h, hkv, t, beg, n;
-};
 
 __device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
   Unit u;
@@ -117,33 +118,43 @@ __device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
 }
 
 // Work queue.  The producer thread claims unit indices from the launch-wide
-// counter p.sched[0] (atomicAdd, longest-first order) and publishes each in a
-// shared-memory ring; the MMA thread and the softmax warps take them from the
-// ring in the same order.  -1 marks the end of the queue.
+// counter p.sched[0] (atomicAdd, longest-first order), decodes each unit and
+// publishes it in a shared-memory ring; the MMA thread, the V loader and the
+// softmax warps take the decoded units from the ring in the same order (so
+// they need no dependent global loads at unit boundaries).  n = -1 marks the
+// end of the queue.
 __device__ __forceinline__ bool publish_unit(const PrefillParams& p, Bars* bars, uint32_t n,
-                                             int* ui) {
+                                             Unit* out) {
   const uint32_t slot = n % kUnitRing;
   if (!wait_bounded(smem_u32(&bars->u_empty[slot]), ((n / kUnitRing) & 1) ^ 1, &bars->abort,
                     p.err, W_PROD_UNIT))
     return false;
-  int v = atomicAdd(p.sched, 1);
-  if (v >= p.n_units) v = -1;
-  reinterpret_cast<volatile int*>(bars->unit_slot)[slot] = v;
+  const int v = atomicAdd(p.sched, 1);
+  Unit u;
+  if (v < p.n_units) {
+    u = get_unit(p, v);
+  } else {
+    u.b = u.h = u.hkv = u.t = u.beg = 0;
+    u.n = -1;
+  }
+  volatile int* d = reinterpret_cast<volatile int*>(&bars->unit_slot[slot]);
+  d[0] = u.b; d[1] = u.h; d[2] = u.hkv; d[3] = u.t; d[4] = u.beg; d[5] = u.n;
   mbar_arrive(smem_u32(&bars->u_full[slot]));
-  *ui = v;
+  *out = u;
   return true;
 }
 
-// Consumer side: one thread (MMA) or every lane of a softmax warp calls it;
-// the slot is released once per caller group (the warp's lane 0 after the
-// whole warp has read it).
-__device__ __forceinline__ bool take_unit(const PrefillParams& p, Bars* bars, uint32_t n, int* ui,
+// Consumer side: one thread (MMA, V loader) or every lane of a softmax warp
+// calls it; the slot is released once per caller group (the warp's lane 0
+// after the whole warp has read it).
+__device__ __forceinline__ bool take_unit(const PrefillParams& p, Bars* bars, uint32_t n, Unit* out,
                                           int where, bool whole_warp) {
   const uint32_t slot = n % kUnitRing;
   if (!wait_bounded(smem_u32(&bars->u_full[slot]), (n / kUnitRing) & 1, &bars->abort, p.err,
                     where))
     return false;
-  *ui = reinterpret_cast<volatile int*>(bars->unit_slot)[slot];
+  const volatile int* d = reinterpret_cast<const volatile int*>(&bars->unit_slot[slot]);
+  out->b = d[0]; out->h = d[1]; out->hkv = d[2]; out->t = d[3]; out->beg = d[4]; out->n = d[5];
   if (whole_warp) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&bars->u_empty[slot]));
@@ -162,10 +173,9 @@ __device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars)
   const uint32_t sK = smem_u32(smem + C::OFF_K);
   uint32_t qc = 0, kc = 0;
   for (uint32_t n = 0;; ++n) {
-    int ui;
-    if (!publish_unit(p, bars, n, &ui)) goto drain;
-    if (ui < 0) break;
-    const Unit u = get_unit(p, ui);
+    Unit u;
+    if (!publish_unit(p, bars, n, &u)) goto drain;
+    if (u.n < 0) break;
     if (u.n == 0) continue;
     if (!wait_bounded(smem_u32(&bars->q_empty), (qc & 1) ^ 1, abort_flag, p.err, W_PROD_Q))
       goto drain;
@@ -209,10 +219,9 @@ __device__ void vloader_role(const PrefillParams& p, uint8_t* smem, Bars* bars) 
   const uint32_t sV = smem_u32(smem + C::OFF_V);
   uint32_t vc = 0, g = 0;
   for (uint32_t n = 0;; ++n) {
-    int ui;
-    if (!take_unit(p, bars, n, &ui, W_VL_UNIT, false)) goto drain;
-    if (ui < 0) break;
-    const Unit u = get_unit(p, ui);
+    Unit u;
+    if (!take_unit(p, bars, n, &u, W_VL_UNIT, false)) goto drain;
+    if (u.n < 0) break;
     for (int k = 0; k < u.n; ++k, ++g) {
       bool keep = true;
       if (p.gate) {
@@ -266,13 +275,12 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
   bool ok = true;
 
   for (uint32_t n = 0; ok; ++n) {
-    int ui;
-    if (!take_unit(p, bars, n, &ui, W_MMA_UNIT, false)) {
+    Unit u;
+    if (!take_unit(p, bars, n, &u, W_MMA_UNIT, false)) {
       ok = false;
       break;
     }
-    if (ui < 0) break;
-    const Unit u = get_unit(p, ui);
+    if (u.n < 0) break;
     if (u.n == 0) continue;
     if (!wait_bounded(smem_u32(&bars->q_full), qc & 1, abort_flag, p.err, W_MMA_Q)) {
       ok = false;
@@ -513,10 +521,9 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
   uint32_t g = 0, pv_total = 0;
 
   for (uint32_t n = 0;; ++n) {
-    int ui;
-    if (!take_unit(p, bars, n, &ui, W_SM_UNIT, true)) return;
-    if (ui < 0) break;
-    const Unit u = get_unit(p, ui);
+    Unit u;
+    if (!take_unit(p, bars, n, &u, W_SM_UNIT, true)) return;
+    if (u.n < 0) break;
     const int i = u.t * kTileQ + row;
     const bool row_ok = i < p.N;
     const int64_t orow = ((int64_t)(u.b * p.H + u.h) * p.N + i);
