@@ -26,7 +26,8 @@ import numpy as np
 from ._lib import (EXPORTS, LIB_PATH, SA_ERR_DEVICE_INDEX, SA_ERR_INVALID_ARG, SA_ERR_TIMEOUT,
                    SA_ERR_UNSUPPORTED, SA_OK, SaPattern, SaPlanInfo, SparseAttnError, check, lib)
 
-__all__ = ["Pattern", "Plan", "sparse_attn_prefill", "sparse_attn_prefill_noalloc",
+__all__ = ["Pattern", "Plan", "KERNEL_AUTO", "KERNEL_SINGLE_HEAD", "KERNEL_PAIRED_HEADS",
+           "sparse_attn_prefill", "sparse_attn_prefill_noalloc",
            "sparse_attn_gather", "compile_pattern",
            "check_device_error", "SparseAttnError", "EXPORTS", "LIB_PATH", "SA_OK",
            "SA_ERR_INVALID_ARG", "SA_ERR_UNSUPPORTED", "SA_ERR_TIMEOUT", "SA_ERR_DEVICE_INDEX"]
@@ -81,14 +82,25 @@ def _check_tensor(name, t, shape, dtype):
     del torch
 
 
-class Plan:
-    """A compiled pattern for Q [B][H][N][d], K/V [B][H_kv][N][d]."""
+KERNEL_AUTO = 0            # the kernel measured fastest for the shape (single-head today)
+KERNEL_SINGLE_HEAD = 1     # the single-head kernel
+KERNEL_PAIRED_HEADS = 2    # the paired-head kernel (d=128, even GQA group, no random table)
 
-    def __init__(self, pattern: Pattern, B: int, H: int, H_kv: int, N: int, d: int):
+
+class Plan:
+    """A compiled pattern for Q [B][H][N][d], K/V [B][H_kv][N][d].
+
+    ``kernel``: KERNEL_AUTO, KERNEL_SINGLE_HEAD or KERNEL_PAIRED_HEADS
+    (sparse_attn_plan_create_ex); ``info["paired_heads"]`` tells which kernel
+    the plan runs on."""
+
+    def __init__(self, pattern: Pattern, B: int, H: int, H_kv: int, N: int, d: int,
+                 kernel: int = KERNEL_AUTO):
         self.pattern, self.B, self.H, self.H_kv, self.N, self.d = pattern, B, H, H_kv, N, d
         st, _tab = pattern.to_c()
         h = ctypes.c_void_p()
-        check(lib().sparse_attn_plan_create(ctypes.byref(st), B, H, H_kv, N, d, ctypes.byref(h)))
+        check(lib().sparse_attn_plan_create_ex(ctypes.byref(st), B, H, H_kv, N, d, kernel,
+                                               ctypes.byref(h)))
         self._h = h
         info = SaPlanInfo()
         check(lib().sparse_attn_plan_info(self._h, ctypes.byref(info)))

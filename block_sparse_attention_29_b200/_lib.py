@@ -22,7 +22,8 @@ SA_ERR_DEVICE_INDEX = 6
 
 # Every function the header declares (tests check the library exports them all).
 EXPORTS = (
-    "sparse_attn_plan_create", "sparse_attn_plan_info", "sparse_attn_plan_destroy",
+    "sparse_attn_plan_create", "sparse_attn_plan_create_ex", "sparse_attn_plan_info",
+    "sparse_attn_plan_destroy",
     "sparse_attn_prefill_plan", "sparse_attn_prefill", "sparse_attn_block_stats",
     "sparse_attn_calibrate", "sparse_attn_gather", "sparse_attn_compile_pattern",
     "sparse_attn_check_device_error", "sparse_attn_last_error", "sparse_attn_prefill_noalloc",
@@ -44,7 +45,8 @@ class SaPlanInfo(ctypes.Structure):
     _fields_ = [("T_q", ctypes.c_int32), ("n_kb", ctypes.c_int32),
                 ("n_units", ctypes.c_int64), ("blocks", ctypes.c_int64),
                 ("blocks_full", ctypes.c_int64), ("blocks_desc", ctypes.c_int64),
-                ("pairs", ctypes.c_int64), ("compile_ms", ctypes.c_double)]
+                ("pairs", ctypes.c_int64), ("compile_ms", ctypes.c_double),
+                ("paired_heads", ctypes.c_int32)]
 
 
 class SparseAttnError(RuntimeError):
@@ -68,6 +70,8 @@ def lib():
                                   ctypes.c_float, ctypes.c_double)
         P = ctypes.POINTER(SaPattern)
         L.sparse_attn_plan_create.argtypes = [P, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]
+        L.sparse_attn_plan_create_ex.argtypes = [P, i32, i32, i32, i32, i32, i32,
+                                                 ctypes.POINTER(vp)]
         L.sparse_attn_plan_info.argtypes = [vp, ctypes.POINTER(SaPlanInfo)]
         L.sparse_attn_plan_destroy.argtypes = [vp]
         L.sparse_attn_plan_destroy.restype = None

@@ -114,6 +114,7 @@ struct sa_plan {
   int B = 0, H = 0, Hkv = 0, N = 0, d = 0, device = 0;
   int T = 0, n_kb = 0, H_pat = 0;
   int n_units = 0;
+  bool pair = false;           // paired-head kernel (units are head pairs)
   int32_t* d_row_ptr = nullptr;
   int32_t* d_entries = nullptr;
   int32_t* d_units = nullptr;
@@ -216,6 +217,7 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
   p->rtab = plan->d_rtab;
   p->thresholds = thresholds;
   p->n_units = plan->n_units;
+  p->pair = plan->pair ? 1 : 0;
   p->B = plan->B;
   p->H = plan->H;
   p->Hkv = plan->Hkv;
@@ -264,7 +266,15 @@ int sparse_attn_compile_pattern(const sa_pattern_t* pat, int H, int N, int tile_
 
 int sparse_attn_plan_create(const sa_pattern_t* pat, int B, int H, int H_kv, int N, int d,
                             sa_plan_t** out) {
+  return sparse_attn_plan_create_ex(pat, B, H, H_kv, N, d, SA_KERNEL_AUTO, out);
+}
+
+int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, int N, int d,
+                               int kernel, sa_plan_t** out) {
   if (!out) return set_error(SA_ERR_INVALID_ARG, "out is NULL");
+  if (kernel != SA_KERNEL_AUTO && kernel != SA_KERNEL_SINGLE_HEAD &&
+      kernel != SA_KERNEL_PAIRED_HEADS)
+    return set_error(SA_ERR_INVALID_ARG, "kernel = %d (not an SA_KERNEL_* value)", kernel);
   *out = nullptr;
   int rc = check_shapes(pat, B, H, H_kv, N, d);
   if (rc) return rc;
@@ -272,6 +282,10 @@ int sparse_attn_plan_create(const sa_pattern_t* pat, int B, int H, int H_kv, int
   CompiledPattern cp;
   rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
   if (rc) return rc;
+  if (kernel == SA_KERNEL_PAIRED_HEADS && !pair_kernel_fits(d, H, H_kv, cp.H_pat))
+    return set_error(SA_ERR_UNSUPPORTED,
+                     "the paired-head kernel needs d = 128, an even number of query heads per "
+                     "K/V head and no random table");
 
   sa_plan_t* plan = new sa_plan_t;
   plan->pat = *pat;
@@ -315,9 +329,11 @@ int sparse_attn_plan_create(const sa_pattern_t* pat, int B, int H, int H_kv, int
     plan->info.blocks_desc = int64_t(cd.kb.size()) * int64_t(B) * (cd.H_pat == 1 ? H : 1);
   }
 
-  plan->n_units = B * cp.T * H;
+  plan->pair = kernel == SA_KERNEL_PAIRED_HEADS;
+  plan->info.paired_heads = plan->pair ? 1 : 0;
+  plan->n_units = B * cp.T * (plan->pair ? H / 2 : H);
   std::vector<int32_t> units;
-  order_units(cp, B, H, H_kv, int64_t(B) * H_kv * N * d * 2 * 2, &units);
+  build_units(cp, B, H, H_kv, N, d, plan->pair, &units);
 
   rc = upload(&plan->d_row_ptr, cp.row_ptr.data(), cp.row_ptr.size());
   if (!rc) rc = upload(&plan->d_entries, entries.data(), entries.size());

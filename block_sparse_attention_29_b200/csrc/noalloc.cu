@@ -92,7 +92,8 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   int rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
   if (rc) return rc;
   const int T = cp.T;
-  const int64_t n_units = int64_t(B) * H * T;
+  const bool pair = false;   // the single-head kernel (the default of the plan API)
+  const int64_t n_units = int64_t(B) * (pair ? H / 2 : H) * T;
   const int nrb = rnd ? (N + pat->random_block - 1) / pat->random_block : 0;
   const size_t b_row = round256(cp.row_ptr.size() * 4);
   const size_t b_ent = round256(std::max<size_t>(cp.kb.size(), 1) * 4);
@@ -109,7 +110,7 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   std::vector<int32_t> entries(cp.kb.size());
   for (size_t e = 0; e < cp.kb.size(); ++e) entries[e] = entry_pack(cp.kb[e], !cp.full[e]);
   std::vector<int32_t> units;
-  order_units(cp, B, H, H_kv, int64_t(B) * H_kv * N * d * 2 * 2, &units);
+  build_units(cp, B, H, H_kv, N, d, pair, &units);
 
   unsigned char* base = nullptr;
   rc = scratch_address(&base);
@@ -151,6 +152,7 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   p.rtab = d_rtab;
   p.thresholds = pat->thresholds;
   p.n_units = int(n_units);
+  p.pair = pair ? 1 : 0;
   p.B = B;
   p.H = H;
   p.Hkv = H_kv;

@@ -151,7 +151,7 @@ int compile_pattern(const sa_pattern_t* p, int H, int N, int tile_q, int tile_k,
   return SA_OK;
 }
 
-void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_bytes,
+void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_bytes, int ctas,
                  std::vector<int32_t>* out) {
   const int T = cp.T;
   const int64_t n = int64_t(B) * H * T;
@@ -165,17 +165,17 @@ void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_b
   };
   int64_t total = 0;
   for (int64_t u = 0; u < n; ++u) total += cost(int32_t(u));
-  // Units longer than half of one CTA's share of the work (2 CTAs per SM on
-  // a 148-SM part) would set the tail if they started late: they go first,
+  // Units longer than half of one CTA's share of the work would set the tail
+  // if they started late: they go first,
   // longest first.  When all of K and V fit in half of L2 the rest are
   // ordered tile-major (later tiles first, the larger ones under a causal
   // mask); otherwise K/V-group-major -- all tiles of the query heads that
   // share one K/V head run together, so that head's K and V stay in L2 while
   // they are reused -- longest first inside a group.  The query heads of a
   // group are adjacent either way.
-  const int64_t heavy = std::max<int64_t>(1, total / (2 * 296) / 2);
+  const int64_t heavy = std::max<int64_t>(1, total / (2 * std::max(ctas, 1)) / 2);
   const bool group_major = kv_bytes > (int64_t(64) << 20);
-  const int group = H / H_kv;
+  const int group = std::max(H / H_kv, 1);
   std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
     const int ca = cost(a), cb = cost(b);
     const bool ha_ = ca > heavy, hb_ = cb > heavy;

@@ -37,6 +37,7 @@
 
 #include "common.h"
 #include "ptx.cuh"
+#include "softmax_util.cuh"
 
 namespace sa {
 namespace {
@@ -383,132 +384,6 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
   }
 }
 
-// --------------------------------------------------------------- softmax --
-// Maximum over the 32 lanes of a warp (one redux instruction on sm_100a).
-__device__ __forceinline__ float warp_max(float v) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
-
-// Bits [lo, hi) of a 64-bit mask, with lo and hi clamped to [0, 64].
-__device__ __forceinline__ uint64_t range_bits(int lo, int hi) {
-  lo = max(lo, 0);
-  hi = min(hi, 64);
-  if (hi <= lo) return 0ull;
-  const uint64_t upto_hi = hi >= 64 ? ~0ull : ((1ull << hi) - 1ull);
-  return upto_hi & ~((1ull << lo) - 1ull);
-}
-
-// A row's random key blocks, read once per work unit (the row's random-block
-// row does not change inside a unit): up to kRowRandom held in registers,
-// longer lists read from global memory.
-constexpr int kRowRandom = 3;
-struct RowRandom {
-  int n;
-  int v[kRowRandom];
-  const int32_t* row;
-};
-
-__device__ __forceinline__ RowRandom load_row_random(const PrefillParams& p, int h, int i) {
-  RowRandom rr;
-  rr.n = 0;
-  rr.row = nullptr;
-  if (p.n_random > 0 && i < p.N) {
-    const int nrb = (p.N + p.random_block - 1) / p.random_block;
-    rr.row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
-    rr.n = p.n_random;
-#pragma unroll
-    for (int r = 0; r < kRowRandom; ++r) rr.v[r] = r < rr.n ? __ldg(rr.row + r) : -1;
-  }
-  return rr;
-}
-
-// Visible keys of row i inside block kb, as a 64-bit mask (bit c = key
-// kb*64 + c).  Every primitive is one index range per row (random blocks cover
-// whole 64-key blocks), so the union is built from ranges; the causal cap and
-// the sequence end are applied last.  Same predicate as the pattern compiler.
-__device__ __forceinline__ uint64_t visible_bits(const PrefillParams& p, const RowRandom& rr,
-                                                 int i, int kb) {
-  if (i >= p.N) return 0ull;
-  const int j0 = kb * kTileK;
-  const bool any_prim = p.window > 0 || p.n_global > 0 || p.block_local > 0 || p.n_random > 0;
-  uint64_t m = 0ull;
-  if (!any_prim || i < p.n_global) {
-    m = ~0ull;
-  } else {
-    if (p.n_global > 0) m |= range_bits(0, p.n_global - j0);
-    if (p.window > 0) {
-      if (p.causal) m |= range_bits(i - p.window + 1 - j0, i + 1 - j0);
-      else m |= range_bits(i - p.window / 2 - j0, i + p.window / 2 + 1 - j0);
-    }
-    if (p.block_local > 0) {
-      const int lo = (i / p.block_local) * p.block_local;
-      m |= range_bits(lo - j0, lo + p.block_local - j0);
-    }
-    if (rr.n > 0) {
-      const int kr = j0 / p.random_block;
-      bool rnd = false;
-#pragma unroll
-      for (int r = 0; r < kRowRandom; ++r) rnd |= rr.v[r] == kr;
-      for (int r = kRowRandom; r < rr.n; ++r) rnd |= __ldg(rr.row + r) == kr;
-      if (rnd) m = ~0ull;
-    }
-  }
-  if (p.causal) m &= range_bits(0, i + 1 - j0);
-  m &= range_bits(0, p.N - j0);
-  return m;
-}
-
-// x[c] = -inf where bit c of the visibility mask is clear.
-__device__ __forceinline__ void apply_mask(uint64_t m, float (&x)[64]) {
-  const uint32_t lo = static_cast<uint32_t>(m), hi = static_cast<uint32_t>(m >> 32);
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    if (!((lo >> c) & 1u)) x[c] = -INFINITY;
-    if (!((hi >> c) & 1u)) x[32 + c] = -INFINITY;
-  }
-}
-
-// ---- softmax arithmetic on 64 logits per thread ----
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// Row maximum as a tree of 3-input maxima (depth 4 instead of a 63-long chain).
-__device__ __forceinline__ float row_max64(const float (&x)[64]) {
-  float a[22];
-#pragma unroll
-  for (int k = 0; k < 21; ++k) a[k] = max3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
-  a[21] = x[63];
-  float b[8];
-#pragma unroll
-  for (int k = 0; k < 7; ++k) b[k] = max3(a[3 * k], a[3 * k + 1], a[3 * k + 2]);
-  b[7] = a[21];
-  return max3(max3(b[0], b[1], b[2]), max3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
-}
-
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 template <int D>
 __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, int warp,
                              int lane) {
@@ -788,6 +663,7 @@ bool g_attr_set[2][64] = {{false}};
 }  // namespace
 
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream) {
+  if (p.pair) return launch_prefill_pair(p, d, stream);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");

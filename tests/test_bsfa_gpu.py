@@ -27,8 +27,9 @@ def _tensors(w, device):
     return Q.to(device), K.to(device), V.to(device)
 
 
-@pytest.mark.parametrize("d", [128, 64])
-def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d):
+@pytest.mark.parametrize("d,kernel", [(128, 0), (128, 2), (64, 0)],
+                         ids=["d128", "d128-paired", "d64"])
+def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d, kernel):
     w = _small(d=d)
     Qc, Kc, Vc, _ = calibration_inputs(w, device="cpu")
     opat = oracle_mod.Pattern(**w.pattern_fields())
@@ -37,7 +38,9 @@ def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d):
     # the same (rounded) threshold values
     tau = oracle_mod.calibrate_thresholds(full_c, stat_c).astype(np.float32).astype(np.float64)
     Q, K, V = _tensors(w, cuda)
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
+                        kernel=kernel)
+    assert plan.info["paired_heads"] == int(kernel == 2)
     tau_d = torch.tensor(tau, dtype=torch.float32, device=cuda)
     mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
     stat = torch.full((w.B, w.H, plan.T, plan.n_kb), float("-inf"), device=cuda)
@@ -59,10 +62,12 @@ def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d):
     assert_close(lse, lr, what="lse")
 
 
-def test_bsfa_extreme_thresholds(product, oracle_mod, cuda):
+@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
+def test_bsfa_extreme_thresholds(product, oracle_mod, cuda, kernel):
     w = _small(N=768, H=2, Hkv=1)
     Q, K, V = _tensors(w, cuda)
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
+                        kernel=kernel)
     mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
     # -inf: nothing skipped, equals the static causal path bit for bit
     O_static = plan.prefill(Q, K, V)
@@ -90,11 +95,13 @@ def test_bsfa_extreme_thresholds(product, oracle_mod, cuda):
     assert_close(O_pinf, Or)
 
 
-def test_device_calibration_matches_oracle(product, oracle_mod, cuda):
+@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
+def test_device_calibration_matches_oracle(product, oracle_mod, cuda, kernel):
     """Statistics pass + per-head rank selection on the GPU == oracle calibration."""
     w = _small(N=1024, H=4, Hkv=2)
     Qc, Kc, _, _ = calibration_inputs(w, device="cpu")
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
+                        kernel=kernel)
     stat = plan.block_stats(Qc.to(cuda), Kc.to(cuda))
     tau_gpu = plan.calibrate(stat, 0.5).cpu().numpy()
     opat = oracle_mod.Pattern(**w.pattern_fields())
@@ -110,11 +117,13 @@ def test_device_calibration_matches_oracle(product, oracle_mod, cuda):
 
 
 @pytest.mark.slow
-def test_bsfa_full_size_sampled(product, oracle_mod, cuda):
+@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
+def test_bsfa_full_size_sampled(product, oracle_mod, cuda, kernel):
     """bsfa_causal at N=32768: device calibration on the calibration draw, then the
     rule; masks checked on sampled tiles, outputs on sampled rows."""
     w = WORKLOADS["bsfa_causal"]
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
+                        kernel=kernel)
     Qc, Kc, _, _ = calibration_inputs(w, device=cuda)
     tau_d = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
     del Qc, Kc
@@ -160,3 +169,27 @@ def test_bsfa_full_size_sampled(product, oracle_mod, cuda):
     Or, _ = oracle_mod.prefill(opat, Qh, Kh, Vh, thresholds=tau, rows=rows, override=override)
     sel = tuple(torch.from_numpy(rows[:, k]).long() for k in range(3))
     assert_close(O.cpu()[sel], Or)
+
+
+@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
+@pytest.mark.parametrize("tau_kind", ["calibrated", "plus_inf"])
+def test_bsfa_repeated_launches_stable(product, oracle_mod, cuda, tau_kind, kernel):
+    """Many launches of the rule without block outputs (the timing of the
+    benchmark loop), including pairs of key blocks that both heads skip: no
+    pipeline wait may run out and every launch gives the same bytes."""
+    w = _small(N=4096, H=8, Hkv=2)
+    Q, K, V = _tensors(w, cuda)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
+                        kernel=kernel)
+    if tau_kind == "calibrated":
+        Qc, Kc, _, _ = calibration_inputs(w, device=cuda)
+        tau = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
+    else:
+        tau = torch.full((w.H,), float("inf"), device=cuda)
+    O0 = plan.prefill(Q, K, V, thresholds=tau)
+    product.check_device_error()
+    O = torch.empty_like(O0)
+    for _ in range(40):
+        plan.prefill(Q, K, V, O=O, thresholds=tau)
+        product.check_device_error()
+        assert torch.equal(O, O0)
