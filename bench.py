@@ -215,7 +215,8 @@ def setup_prefill(w, device, torch, sa, workloads):
     return dict(step=step, e2e_step=lambda s: e2e_step(host, dev_bufs, s), h2d=h2d, d2h=d2h,
                 flops=computed, exact_flops=exact, dense_flops=dense, algo_bytes=algo_bytes,
                 extra=extra, kernel="prefill_kernel",
-                kernel_files=["prefill_sm100.cu", "pattern_compiler.cu"],
+                kernel_files=["prefill_sm100.cu", "softmax_util.cuh", "ptx.cuh", "common.h",
+                              "pattern_compiler.cu"],
                 metric="effective TFLOP/s (computed blocks)", unit="TFLOP/s", bound="tensor",
                 tensors=(Q, K, V, O), plan=plan, tab=tab, thresholds=thresholds)
 
