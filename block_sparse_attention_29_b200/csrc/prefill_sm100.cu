@@ -26,11 +26,12 @@
 // them) and each CTA's producer claims the next one with an atomic counter
 // when it has room, so CTAs that get cheap units take more of them.
 //
-// TMEM columns: S at [0, 64), P buffers at [64, 96) and [96, 128) (bf16
-// pairs), O at [128, 128 + d).  S has one buffer: the next block's QK^T is
-// issued as soon as the softmax warps have loaded the current S into
-// registers, so it overlaps their exponentials; P has two, so the PV of one
-// block and the P of the next do not wait for each other.
+// TMEM columns: two S buffers at [0, 64) and [64, 128), O at [128, 128 + d).
+// Block k uses S buffer k % 2; its P (bf16 pairs) is written over the first
+// 32 columns of that buffer once the logits are in registers, and the PV of
+// block k reads it there.  The QK^T of block k+1 runs while the softmax works
+// on block k, also when block k is skipped by the rule, so a run of skipped
+// blocks costs the softmax's statistic alone per block.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -44,8 +45,7 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
-constexpr int kTmemS = 0;     // S of the current block: 64 fp32 columns
-constexpr int kTmemP = 64;    // two P buffers of 32 columns (64 bf16 per row)
+constexpr int kTmemS = 0;     // two S buffers of 64 fp32 columns, at kTmemS + 64 b
 constexpr int kTmemO = 128;   // O accumulator: d fp32 columns
 constexpr uint32_t kSoftmaxBar = 1;    // named barrier of the softmax warpgroup
 constexpr uint32_t kSoftmaxWarps = 4;
@@ -87,10 +87,9 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[3], k_empty[3];
   uint64_t v_full[3], v_empty[3];
-  uint64_t s_full, s_free;              // the single S buffer: written / read out
+  uint64_t s_full[2];                   // per S buffer: S of the block written
   uint64_t p_ready[2];                  // per block parity: P written (or block skipped)
   uint64_t dec_full[4], dec_empty[4];   // gate decisions, softmax -> V loader
-  uint64_t p_free[2];                   // per P buffer: the PV that read it is done
   uint64_t o_done[2];
   uint64_t drain;
   uint64_t u_full[4], u_empty[4];   // work-unit ring (producer -> MMA + softmax)
@@ -258,8 +257,11 @@ drain:
 // ----------------------------------------------------------- MMA issuer --
 // One thread, an event loop per work unit that never blocks on one condition
 // while another step is ready.  Steps, each issued in block order:
-//   S  : S_k = Q K_k^T once the softmax has read S_{k-1} out of TMEM and K_k
-//        is in shared memory (and at most one block ahead of the P hand-off);
+//   S  : S_k = Q K_k^T into S buffer k % 2 once K_k is in shared memory and
+//        block k-2, the buffer's previous user, is done: its hand-off taken
+//        and, if kept, its PV issued (the PV reads P_{k-2} from that buffer
+//        and is issued first; tcgen05.mma operations of one thread execute
+//        in issue order);
 //   P  : take block k's P hand-off (kept or skipped) from the softmax;
 //   PV : O += P_k V_k for a kept block once V_k has landed.
 template <int D>
@@ -298,21 +300,20 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
     while (npv < u.n) {
       bool progress = false;
       // S for block ns.
-      if (ns < u.n && ns <= nr + 1) {
+      if (ns < u.n && ns <= npv + 1) {
         const uint32_t st = kc % C::KS;
-        if (mbar_try_wait(smem_u32(&bars->s_free), ((g0 + ns) & 1) ^ 1) &&
-            mbar_try_wait(smem_u32(&bars->k_full[st]), (kc / C::KS) & 1)) {
-          tc_fence_after();
+        if (mbar_try_wait(smem_u32(&bars->k_full[st]), (kc / C::KS) & 1)) {
+          const uint32_t sb = (g0 + ns) & 1;
           const uint32_t kbase = sK + st * C::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk & 3) * 32;
             const uint64_t da = make_sdesc(sQ + (kk >> 2) * (kTileQ * 128) + off, 16, 1024);
             const uint64_t db = make_sdesc(kbase + (kk >> 2) * (kTileK * 128) + off, 16, 1024);
-            umma_ss(tmem + kTmemS, da, db, idesc_s, kk > 0 ? 1u : 0u);
+            umma_ss(tmem + kTmemS + 64 * sb, da, db, idesc_s, kk > 0 ? 1u : 0u);
           }
           tc_commit(smem_u32(&bars->k_empty[st]));
-          tc_commit(smem_u32(&bars->s_full));
+          tc_commit(smem_u32(&bars->s_full[sb]));
           if (ns == u.n - 1) tc_commit(smem_u32(&bars->q_empty));
           ++kc;
           ++g;
@@ -341,7 +342,7 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
           if (mbar_try_wait(smem_u32(&bars->v_full[vs]), (pvc / C::VS) & 1)) {
             tc_fence_after();
             const uint32_t vbase = sV + vs * C::KV_BYTES;
-            const uint32_t pcol = kTmemP + (pvc & 1) * 32;
+            const uint32_t pcol = kTmemS + 64 * ((g0 + npv) & 1);   // P over block npv's S
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
               const uint64_t db = make_sdesc(vbase + kk * (16 * 128), kTileK * 128, 1024);
@@ -349,7 +350,6 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
                       (first_pv && kk == 0) ? 0u : 1u);
             }
             tc_commit(smem_u32(&bars->v_empty[vs]));
-            tc_commit(smem_u32(&bars->p_free[pvc & 1]));
             tc_commit(smem_u32(&bars->o_done[pvc & 1]));
             ++pvc;
             ++npv;
@@ -424,13 +424,17 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       if (leader && p.gate)
         slot_ok = wait_bounded(smem_u32(&bars->dec_empty[g % kDecRing]),
                                ((g / kDecRing) & 1) ^ 1, abort_flag, p.err, W_SM_DEC);
-      if (!wait_bounded(smem_u32(&bars->s_full), g & 1, abort_flag, p.err, W_SM_S)) return;
+      // S of this block is in S buffer fb; the MMA thread computes the next
+      // block's S into the other buffer meanwhile.
+      const uint32_t tS = tmem + lane_base + kTmemS + 64 * fb;
+      if (!wait_bounded(smem_u32(&bars->s_full[fb]), (g >> 1) & 1, abort_flag, p.err, W_SM_S))
+        return;
       tc_fence_after();
       float x[64];
       {
         uint32_t r0[32], r1[32];
-        tmem_ld32(tmem + lane_base + kTmemS, r0);
-        tmem_ld32(tmem + lane_base + kTmemS + 32, r1);
+        tmem_ld32(tS, r0);
+        tmem_ld32(tS + 32, r1);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -438,10 +442,6 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
           x[32 + c] = __uint_as_float(r1[c]);
         }
       }
-      // S is in registers: release the S columns for the next block's QK^T.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_free));
       if (partial) apply_mask(vis, x);
       const float mx = row_max64(x);
 
@@ -449,6 +449,10 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       if (p.want_stats) {
         const float wm = warp_max(mx);
         if (lane == 0) bars->red[fb][q4] = wm;
+        // Past this barrier every warp has read its rows of S (a skipped
+        // block is handed off by the leader alone, after which the MMA thread
+        // may overwrite the buffer).
+        tc_fence_before();
         named_bar_sync(kSoftmaxBar, 128);
         const float tmax = fmaxf(fmaxf(bars->red[fb][0], bars->red[fb][1]),
                                  fmaxf(bars->red[fb][2], bars->red[fb][3]));
@@ -485,12 +489,6 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         l *= alpha;
         m = m_new;
       }
-      // This block's P goes to P buffer (pv_total & 1), free once the PV two
-      // before it has completed; after this wait at most one PV is in flight.
-      const uint32_t pb = pv_total & 1;
-      if (!wait_bounded(smem_u32(&bars->p_free[pb]), ((pv_total >> 1) & 1) ^ 1, abort_flag, p.err,
-                        W_SM_P))
-        return;
       if (kept > 0 && __any_sync(0xffffffffu, need)) {
         // O += P V of the previous kept block must be complete before O is rescaled.
         const uint32_t last = pv_total - 1;
@@ -532,7 +530,9 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
         l += s0 + s1;
       }
-      tmem_st32(tmem + lane_base + kTmemP + pb * 32, pk);
+      // P (bf16 pairs) over the first 32 columns of this block's S buffer,
+      // whose logits are in registers.
+      tmem_st32(tS, pk);
       tmem_wait_st();
       tc_fence_before();
       // Each warp signals its own 32 rows of P; the MMA warp waits for all four.
@@ -599,10 +599,8 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
       mbar_init(smem_u32(&bars->v_full[s]), 1);
       mbar_init(smem_u32(&bars->v_empty[s]), 1);
     }
-    mbar_init(smem_u32(&bars->s_full), 1);
-    mbar_init(smem_u32(&bars->s_free), kSoftmaxWarps);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&bars->p_free[b]), 1);
+      mbar_init(smem_u32(&bars->s_full[b]), 1);
       mbar_init(smem_u32(&bars->p_ready[b]), kSoftmaxWarps);
       mbar_init(smem_u32(&bars->o_done[b]), 1);
     }
