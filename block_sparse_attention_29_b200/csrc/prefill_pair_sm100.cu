@@ -515,8 +515,16 @@ __device__ void softmax2(const PrefillParams& p, Bars2* bars, uint32_t tmem, int
       const int kba = ea >> 1, kbb = eb >> 1;
       const bool pa = ea & 1, pb = eb & 1;
       uint64_t visa = ~0ull, visb = ~0ull;
-      if (pa) visa = visible_bits_static(p, i, kba);
-      if (pb) visb = visible_bits_static(p, i, kbb);
+      if (pa || pb) {
+        // The paired-head kernel never sees random tables; the row's part of
+        // the predicate is cheap enough to build per partial pair.
+        RowRandom none;
+        none.n = 0;
+        none.row = nullptr;
+        const RowVis rv = row_vis(p, none, i);
+        if (pa) visa = vis_bits(p, rv, h, i, kba);
+        if (pb) visb = vis_bits(p, rv, h, i, kbb);
+      }
       bool slot_ok = true;
       if (leader && post_dec)
         slot_ok = wait_bounded(smem_u32(&bars->dec_empty[x][g % kDecRing2]),

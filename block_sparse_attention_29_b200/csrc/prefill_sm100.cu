@@ -408,7 +408,7 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
     uint32_t kept = 0;
     // Block entries are read one block ahead so the load overlaps the S wait.
     int e_next = u.n > 0 ? __ldg(p.entries + u.beg) : 0;
-    const RowRandom rr = load_row_random(p, u.h, i);
+    const RowVis rv = row_vis(p, load_row_random(p, u.h, i), i);
 
     for (int k = 0; k < u.n; ++k) {
       const uint32_t fb = g & 1;   // per-block-parity flag / decision slot
@@ -417,7 +417,7 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       const int kb = e >> 1;
       const bool partial = e & 1;
       uint64_t vis = ~0ull;
-      if (partial) vis = visible_bits(p, rr, i, kb);
+      if (partial) vis = vis_bits(p, rv, u.h, i, kb);
       // The leader claims this block's decision-ring slot now, while S is
       // still being computed (the V loader frees slots as it reads them).
       bool slot_ok = true;
@@ -442,7 +442,7 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
           x[32 + c] = __uint_as_float(r1[c]);
         }
       }
-      if (partial) apply_mask(vis, x);
+      if (partial && vis != ~0ull) apply_mask(vis, x);
       const float mx = row_max64(x);
 
       bool keep = true;

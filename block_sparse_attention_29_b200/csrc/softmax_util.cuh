@@ -53,60 +53,57 @@ __device__ __forceinline__ RowRandom load_row_random(const PrefillParams& p, int
 // kb*64 + c).  Every primitive is one index range per row (random blocks cover
 // whole 64-key blocks), so the union is built from ranges; the causal cap and
 // the sequence end are applied last.  Same predicate as the pattern compiler.
-__device__ __forceinline__ uint64_t visible_bits(const PrefillParams& p, const RowRandom& rr,
-                                                 int i, int kb) {
-  if (i >= p.N) return 0ull;
-  const int j0 = kb * kTileK;
+// The per-row part (window start, cap, the row's random blocks as the first
+// 64-key block of their range) is computed once per work unit by row_vis, so
+// a block's mask costs a few range masks and compares and no division.
+struct RowVis {
+  int all;              // the row sees every key below cap_hi (global row, or no primitive)
+  int win_lo;           // window keys [win_lo, win_lo + window length)
+  int cap_hi;           // causal cap and sequence end: keys < cap_hi (0 for rows past N)
+  int rlo[kRowRandom];  // the row's first random blocks, as their first 64-key block
+};
+
+__device__ __forceinline__ RowVis row_vis(const PrefillParams& p, const RowRandom& rr, int i) {
+  RowVis v;
   const bool any_prim = p.window > 0 || p.n_global > 0 || p.block_local > 0 || p.n_random > 0;
-  uint64_t m = 0ull;
-  if (!any_prim || i < p.n_global) {
-    m = ~0ull;
-  } else {
-    if (p.n_global > 0) m |= range_bits(0, p.n_global - j0);
+  v.all = (!any_prim || i < p.n_global) ? 1 : 0;
+  v.win_lo = p.causal ? i - p.window + 1 : i - p.window / 2;
+  v.cap_hi = i >= p.N ? 0 : (p.causal ? i + 1 : p.N);
+  const int rb64 = p.random_block / kTileK;
+#pragma unroll
+  for (int r = 0; r < kRowRandom; ++r) v.rlo[r] = r < rr.n ? rr.v[r] * rb64 : -(1 << 30);
+  return v;
+}
+
+__device__ __forceinline__ uint64_t vis_bits(const PrefillParams& p, const RowVis& v, int h,
+                                             int i, int kb) {
+  const int j0 = kb * kTileK;
+  uint64_t m = ~0ull;
+  if (!v.all) {
+    m = range_bits(0, p.n_global - j0);
     if (p.window > 0) {
-      if (p.causal) m |= range_bits(i - p.window + 1 - j0, i + 1 - j0);
-      else m |= range_bits(i - p.window / 2 - j0, i + p.window / 2 + 1 - j0);
+      const int len = p.causal ? p.window : 2 * (p.window / 2) + 1;
+      m |= range_bits(v.win_lo - j0, v.win_lo + len - j0);
     }
     if (p.block_local > 0) {
       const int lo = (i / p.block_local) * p.block_local;
       m |= range_bits(lo - j0, lo + p.block_local - j0);
     }
-    if (rr.n > 0) {
-      const int kr = j0 / p.random_block;
+    if (p.n_random > 0) {
+      const unsigned rb64 = static_cast<unsigned>(p.random_block / kTileK);
       bool rnd = false;
 #pragma unroll
-      for (int r = 0; r < kRowRandom; ++r) rnd |= rr.v[r] == kr;
-      for (int r = kRowRandom; r < rr.n; ++r) rnd |= __ldg(rr.row + r) == kr;
+      for (int r = 0; r < kRowRandom; ++r) rnd |= static_cast<unsigned>(kb - v.rlo[r]) < rb64;
+      if (p.n_random > kRowRandom && i < p.N) {   // longer lists: read from the table
+        const int nrb = (p.N + p.random_block - 1) / p.random_block;
+        const int32_t* row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
+        for (int r = kRowRandom; r < p.n_random; ++r)
+          rnd |= static_cast<unsigned>(kb - __ldg(row + r) * static_cast<int>(rb64)) < rb64;
+      }
       if (rnd) m = ~0ull;
     }
   }
-  if (p.causal) m &= range_bits(0, i + 1 - j0);
-  m &= range_bits(0, p.N - j0);
-  return m;
-}
-
-// visible_bits for a pattern without random blocks (the lists are then the
-// same for every head): window, global tokens, blockwise, causal cap.
-__device__ __forceinline__ uint64_t visible_bits_static(const PrefillParams& p, int i, int kb) {
-  if (i >= p.N) return 0ull;
-  const int j0 = kb * kTileK;
-  uint64_t m;
-  if (i < p.n_global || (p.window <= 0 && p.n_global <= 0 && p.block_local <= 0)) {
-    m = ~0ull;
-  } else {
-    m = range_bits(0, p.n_global - j0);
-    if (p.window > 0) {
-      const int lo = p.causal ? i - p.window + 1 : i - p.window / 2;
-      const int hi = p.causal ? i + 1 : i + p.window / 2 + 1;
-      m |= range_bits(lo - j0, hi - j0);
-    }
-    if (p.block_local > 0) {
-      const int lo = (i / p.block_local) * p.block_local;
-      m |= range_bits(lo - j0, lo + p.block_local - j0);
-    }
-  }
-  if (p.causal) m &= range_bits(0, i + 1 - j0);
-  return m & range_bits(0, p.N - j0);
+  return m & range_bits(0, v.cap_hi - j0);
 }
 
 // x[OFF + c] = -inf where bit c of the visibility mask is clear.
