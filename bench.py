@@ -253,6 +253,40 @@ def setup_gather(w, device, torch, sa, workloads):
                 tensors=(Q, K, V, idx, O), idx=idx)
 
 
+def setup_window_decode(w, device, torch, sa, workloads):
+    Q, K, V, pos = workloads.window_decode_inputs(w, device=device)
+    O = torch.empty_like(Q)
+    pat = sa.Pattern(causal=1, window=w.window, n_global=w.n_global)
+    n_rows = w.window + w.n_global                  # every query sits past the window
+    # each cached row is needed once per (sequence, K/V head): the query heads
+    # of a group read it again from L2
+    algo_bytes = (w.S * w.H_kv * n_rows * 2 * w.d * 2 + Q.numel() * 2 + O.numel() * 2
+                  + pos.numel() * 4)
+    flops = 4 * w.S * w.H * n_rows * w.d
+
+    def step(stream=None):
+        sa.sparse_attn_decode_window(Q, K, V, pos, pat, O=O, stream=stream)
+
+    host = [Q.cpu().pin_memory(), pos.cpu().pin_memory(),
+            torch.empty(O.shape, dtype=O.dtype, pin_memory=True)]
+    Qd, posd, Od = torch.empty_like(Q), torch.empty_like(pos), torch.empty_like(O)
+
+    def e2e_step(stream):
+        Qd.copy_(host[0], non_blocking=True)
+        posd.copy_(host[1], non_blocking=True)
+        sa.sparse_attn_decode_window(Qd, K, V, posd, pat, O=Od, stream=stream)
+        host[2].copy_(Od, non_blocking=True)
+
+    h2d = host[0].numel() * 2 + host[1].numel() * 4
+    d2h = host[2].numel() * 2
+    return dict(step=step, e2e_step=e2e_step, h2d=h2d, d2h=d2h, flops=flops, exact_flops=flops,
+                dense_flops=flops, algo_bytes=algo_bytes,
+                extra={"rows_per_query": n_rows, "cache_slots": n_rows},
+                kernel="gather_kernel", kernel_files=["gather_sm100.cu"],
+                metric="window decode GB/s", unit="GB/s", bound="hbm",
+                tensors=(Q, K, V, pos, O), pos=pos)
+
+
 # ------------------------------------------------------------- CPU baseline --
 def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
     """Times the fp64 oracle as it stands on the host cores over a bounded sample
@@ -263,6 +297,34 @@ def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
     from block_sparse_attention_29_b200 import workloads
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     g = np.random.default_rng(1234 + sample_seed)
+    if isinstance(w, workloads.WindowDecodeWorkload):
+        # window decode: sampled (sequence, head) queries over the oracle's
+        # gather with the cache slots of their index sets (same rows, same order)
+        Q, K, V, pos = device_tensors
+        group = w.H // w.H_kv
+        rows_of = {}   # (s, kv head) -> its cache rows in key order, gathered once
+
+        def rows(s, hk):
+            if (s, hk) not in rows_of:
+                ix = torch.from_numpy(workloads.window_slots_in_key_order(
+                    int(pos[s]), w.window, w.n_global)).to(K.device)
+                rows_of[(s, hk)] = (K[s, hk, ix].cpu(), V[s, hk, ix].cpu())
+            return rows_of[(s, hk)]
+        done_rows, t_total, n = 0, 0.0, 8
+        while t_total < seconds:
+            pairs = [(int(g.integers(w.S)), int(g.integers(w.H))) for _ in range(n)]
+            Qh = torch.stack([Q[s, h] for s, h in pairs])[None].cpu()
+            Kh = torch.stack([rows(s, h // group)[0] for s, h in pairs])[None]
+            Vh = torch.stack([rows(s, h // group)[1] for s, h in pairs])[None]
+            m = Kh.shape[2]
+            local = np.broadcast_to(np.arange(m, dtype=np.int32), (1, n, m)).copy()
+            t0 = time.perf_counter()
+            oracle.gather(Qh, Kh, Vh, local, nthreads=cores)
+            t_total += time.perf_counter() - t0
+            done_rows += n * m
+            n = min(32, n * 2)
+        gbs = done_rows * (2 * w.d * 2) / t_total / 1e9
+        return gbs, cores, f"{done_rows // m} (sequence, head) queries, {done_rows} cache rows"
     if isinstance(w, workloads.GatherWorkload):
         # gather: sampled (sequence, head) sets, only their referenced rows on the host
         if device_tensors is None:
@@ -351,7 +413,10 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
 
-    setup = setup_gather if isinstance(w, workloads.GatherWorkload) else setup_prefill
+    if isinstance(w, workloads.WindowDecodeWorkload):
+        setup = setup_window_decode
+    else:
+        setup = setup_gather if isinstance(w, workloads.GatherWorkload) else setup_prefill
     S = setup(w, device, torch, sa, workloads)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
@@ -443,7 +508,7 @@ def main():
                             "algorithmic_bytes": S["algo_bytes"], **S["extra"]}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        if isinstance(w, workloads.GatherWorkload):
+        if isinstance(w, (workloads.GatherWorkload, workloads.WindowDecodeWorkload)):
             Q, K, V, idx, _ = S["tensors"]
             dt = (Q, K, V, idx)
         else:
@@ -460,6 +525,12 @@ def main():
 
 def config_of(w, world):
     from block_sparse_attention_29_b200 import workloads
+    if isinstance(w, workloads.WindowDecodeWorkload):
+        return {"workload": w.name, "sequences": w.S, "H": w.H, "H_kv": w.H_kv, "d": w.d,
+                "pattern": {"causal": 1, "window": w.window, "n_global": w.n_global},
+                "cache_slots": w.window + w.n_global, "positions": f"uniform in "
+                f"[{w.window + w.n_global}, {w.max_pos}]",
+                "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}
     if isinstance(w, workloads.GatherWorkload):
         return {"workload": w.name, "sequences": w.S, "H": w.H, "H_kv": w.H_kv, "d": w.d,
                 "cache_len": w.L, "n_idx": w.n_idx, "H_idx": w.H_idx,
@@ -476,7 +547,12 @@ def run_reference(args, w, world):
     oracle.build()
     from block_sparse_attention_29_b200 import workloads
     dt = None
-    if isinstance(w, workloads.GatherWorkload):
+    if isinstance(w, workloads.WindowDecodeWorkload):
+        import dataclasses
+        ws = dataclasses.replace(w, S=4)
+        dt = workloads.window_decode_inputs(ws, device="cpu")
+        w = ws
+    elif isinstance(w, workloads.GatherWorkload):
         # a cache of the full size does not fit the host budget of this arm: the
         # sampled sets' rows are drawn with the same recipe at reduced length
         import dataclasses
@@ -498,8 +574,10 @@ def run_reference(args, w, world):
         vals.append(v)
     elapsed = time.perf_counter() - t0
     value = statistics.mean(vals)
-    unit = "GB/s" if isinstance(w, workloads.GatherWorkload) else "TFLOP/s"
-    metric = "gather GB/s" if unit == "GB/s" else "effective TFLOP/s (computed blocks)"
+    unit = ("GB/s" if isinstance(w, (workloads.GatherWorkload, workloads.WindowDecodeWorkload))
+            else "TFLOP/s")
+    metric = ("window decode GB/s" if isinstance(w, workloads.WindowDecodeWorkload) else
+              "gather GB/s" if unit == "GB/s" else "effective TFLOP/s (computed blocks)")
     out = {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": round(1e3 * elapsed / args.steps, 3), "higher_is_better": True,

@@ -28,7 +28,7 @@ from ._lib import (EXPORTS, LIB_PATH, SA_ERR_DEVICE_INDEX, SA_ERR_INVALID_ARG, S
 
 __all__ = ["Pattern", "Plan", "KERNEL_AUTO", "KERNEL_SINGLE_HEAD", "KERNEL_PAIRED_HEADS",
            "sparse_attn_prefill", "sparse_attn_prefill_noalloc",
-           "sparse_attn_gather", "compile_pattern",
+           "sparse_attn_gather", "sparse_attn_decode_window", "window_slot", "compile_pattern",
            "check_device_error", "SparseAttnError", "EXPORTS", "LIB_PATH", "SA_OK",
            "SA_ERR_INVALID_ARG", "SA_ERR_UNSUPPORTED", "SA_ERR_TIMEOUT", "SA_ERR_DEVICE_INDEX"]
 
@@ -230,6 +230,38 @@ def sparse_attn_gather(Q, K, V, idx, idx_len=None, O=None, scale: float = 0.0, l
                                    S, H, Hkv, H_idx, L, n_idx, d, float(scale), _ptr(lse),
                                    _stream(stream)))
     return O
+
+
+def sparse_attn_decode_window(Q, K, V, positions, pattern: Pattern, O=None, lse=None,
+                              stream=None):
+    """Decode over a minimum-size cache for a causal window + global tokens pattern.
+
+    Q [S][H][d]; K/V [S][H_kv][C][d] with C = window + n_global slots (key j in
+    slot window_slot(j, window, n_global)); positions int32 [S] -> O [S][H][d]."""
+    import torch
+    S, H, d = Q.shape
+    Hkv, C = K.shape[1], K.shape[2]
+    if C != pattern.window + pattern.n_global:
+        raise ValueError(f"cache has {C} slots, the pattern needs window + n_global = "
+                         f"{pattern.window + pattern.n_global}")
+    _check_tensor("Q", Q, (S, H, d), torch.bfloat16)
+    _check_tensor("K", K, (S, Hkv, C, d), torch.bfloat16)
+    _check_tensor("V", V, (S, Hkv, C, d), torch.bfloat16)
+    _check_tensor("positions", positions, (S,), torch.int32)
+    if O is None:
+        O = torch.empty_like(Q)
+    _check_tensor("O", O, (S, H, d), torch.bfloat16)
+    if lse is not None:
+        _check_tensor("lse", lse, (S, H), torch.float32)
+    st, _tab = pattern.to_c()
+    check(lib().sparse_attn_decode_window(_ptr(Q), _ptr(K), _ptr(V), _ptr(positions), _ptr(O), S,
+                                          H, Hkv, d, ctypes.byref(st), _ptr(lse), _stream(stream)))
+    return O
+
+
+def window_slot(j: int, window: int, n_global: int) -> int:
+    """Cache slot of key j in the layout of sparse_attn_decode_window (-1 if invalid)."""
+    return int(lib().sparse_attn_window_slot(int(j), int(window), int(n_global)))
 
 
 def compile_pattern(pattern: Pattern, H: int, N: int, tile_q: int = 128, tile_k: int = 64):

@@ -25,7 +25,8 @@ EXPORTS = (
     "sparse_attn_plan_create", "sparse_attn_plan_create_ex", "sparse_attn_plan_info",
     "sparse_attn_plan_destroy",
     "sparse_attn_prefill_plan", "sparse_attn_prefill", "sparse_attn_block_stats",
-    "sparse_attn_calibrate", "sparse_attn_gather", "sparse_attn_compile_pattern",
+    "sparse_attn_calibrate", "sparse_attn_gather", "sparse_attn_decode_window",
+    "sparse_attn_window_slot", "sparse_attn_compile_pattern",
     "sparse_attn_check_device_error", "sparse_attn_last_error", "sparse_attn_prefill_noalloc",
 )
 
@@ -81,6 +82,9 @@ def lib():
                                                   vp]
         L.sparse_attn_block_stats.argtypes = [vp, vp, vp, vp, vp, vp]
         L.sparse_attn_calibrate.argtypes = [vp, vp, f64, vp, vp]
+        L.sparse_attn_decode_window.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, P, vp, vp]
+        L.sparse_attn_window_slot.argtypes = [i64, i32, i32]
+        L.sparse_attn_window_slot.restype = i64
         L.sparse_attn_gather.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                          i32, f32, vp, vp]
         L.sparse_attn_compile_pattern.argtypes = [P, i32, i32, i32, i32,

@@ -485,11 +485,62 @@ int sparse_attn_gather(const void* Q, const void* K, const void* V, const int32_
   p.H_idx = H_idx;
   p.L = L;
   p.n_idx = n_idx;
+  p.positions = nullptr;
+  p.window = p.n_global = 0;
   const float sc = scale != 0.f ? scale : 1.0f / sqrtf(float(d));
   p.scale_log2 = sc * 1.4426950408889634f;
   p.err = device_error_word();
   if (!p.err) return set_error(SA_ERR_CUDA, "device error word unavailable");
   return launch_gather(p, d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int sparse_attn_decode_window(const void* Q, const void* K, const void* V,
+                              const int32_t* positions, void* O, int S, int H, int H_kv, int d,
+                              const sa_pattern_t* pat, float* lse_out, sa_stream_t stream) {
+  if (!Q || !K || !V || !positions || !O || !pat)
+    return set_error(SA_ERR_INVALID_ARG, "Q, K, V, positions, O and pat must be non-NULL");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return set_error(SA_ERR_INVALID_ARG, "Q, K, V and O must be 16-byte aligned");
+  if (S < 0 || H <= 0 || H_kv <= 0)
+    return set_error(SA_ERR_INVALID_ARG, "bad shape (S=%d H=%d H_kv=%d)", S, H, H_kv);
+  if (H % H_kv != 0) return set_error(SA_ERR_INVALID_ARG, "H = %d is not a multiple of H_kv = %d", H, H_kv);
+  if (d != 64 && d != 128) return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
+  if (!pat->causal || pat->window < 1 || pat->n_global < 0)
+    return set_error(SA_ERR_UNSUPPORTED,
+                     "window decode needs a causal pattern with window >= 1 and n_global >= 0");
+  if (pat->block_local > 0 || (pat->n_random > 0 && pat->random_table) || pat->thresholds)
+    return set_error(SA_ERR_UNSUPPORTED,
+                     "window decode covers the window and global tokens only (no block_local, "
+                     "random blocks or thresholds)");
+  const int64_t C = int64_t(pat->window) + pat->n_global;
+  if (C > INT32_MAX) return set_error(SA_ERR_UNSUPPORTED, "cache of %lld slots too large", (long long)C);
+  GatherParams p;
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.K = static_cast<const uint16_t*>(K);
+  p.V = static_cast<const uint16_t*>(V);
+  p.idx = nullptr;
+  p.idx_len = nullptr;
+  p.O = static_cast<uint16_t*>(O);
+  p.lse = lse_out;
+  p.S = S;
+  p.H = H;
+  p.Hkv = H_kv;
+  p.H_idx = H;
+  p.L = int(C);
+  p.n_idx = 0;
+  p.positions = positions;
+  p.window = pat->window;
+  p.n_global = pat->n_global;
+  const float sc = pat->scale != 0.f ? pat->scale : 1.0f / sqrtf(float(d));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.err = device_error_word();
+  if (!p.err) return set_error(SA_ERR_CUDA, "device error word unavailable");
+  return launch_gather(p, d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int64_t sparse_attn_window_slot(int64_t j, int window, int n_global) {
+  if (j < 0 || window < 1 || n_global < 0) return -1;
+  return j < n_global ? j : n_global + (j % window);
 }
 
 int sparse_attn_check_device_error(sa_stream_t stream) {

@@ -87,6 +87,11 @@ struct GatherParams {
   uint16_t* O;         // [S][H][d]
   float* lse;          // [S][H] or null
   int S, H, Hkv, H_idx, L, n_idx;
+  // Window decode (positions != null): the index set of sequence s is
+  // [0, min(n_global, p+1)) u [max(n_global, p-window+1), p], p = positions[s],
+  // key j in cache slot j (j < n_global) or n_global + (j mod window).
+  const int32_t* positions;
+  int window, n_global;
   float scale_log2;
   int* err;            // device error word
 };

@@ -69,6 +69,22 @@ class GatherWorkload:
     seed: int = 0
 
 
+@dataclass
+class WindowDecodeWorkload:
+    """Decode of a causal window + global tokens pattern over a cache of
+    window + n_global slots; every query sits past the window (its set is the
+    n_global globals and the last `window` keys)."""
+    name: str
+    S: int
+    H: int
+    H_kv: int
+    d: int
+    window: int
+    n_global: int
+    max_pos: int
+    seed: int = 0
+
+
 WORKLOADS = {
     "tiny_static": PrefillWorkload("tiny_static", B=1, H=2, H_kv=2, N=256, d=64, causal=1,
                                    window=64, n_global=4, block_q=64, block_k=64, seed=1000),
@@ -81,6 +97,8 @@ WORKLOADS = {
                                           n_random=3, block_q=128, block_k=64, seed=4000),
     "gather_decode": GatherWorkload("gather_decode", S=64, H=32, H_kv=8, d=128, L=131072,
                                     n_idx=2048, H_idx=32, seed=5000),
+    "window_decode": WindowDecodeWorkload("window_decode", S=64, H=32, H_kv=8, d=128,
+                                          window=4096, n_global=4, max_pos=131071, seed=6000),
 }
 
 
@@ -160,6 +178,27 @@ def gather_inputs(w: GatherWorkload, device="cpu", seed: Optional[int] = None):
     V = randn_bf16((w.S, w.H_kv, w.L, w.d), base + 2, device)
     idx = gather_index_sets(w.S, w.H_idx, w.L, w.n_idx, w.n_recent, base + 3, device)
     return Q, K, V, idx
+
+
+def window_decode_inputs(w: WindowDecodeWorkload, device="cpu", seed: Optional[int] = None):
+    """(Q [S][H][d], K, V [S][H_kv][window + n_global][d] cache, positions int32 [S])
+    with positions uniform in [window + n_global, max_pos] (seeded)."""
+    base = w.seed if seed is None else seed
+    C = w.window + w.n_global
+    Q = randn_bf16((w.S, w.H, w.d), base, device)
+    K = randn_bf16((w.S, w.H_kv, C, w.d), base + 1, device)
+    V = randn_bf16((w.S, w.H_kv, C, w.d), base + 2, device)
+    g = _gen(base + 3, "cpu")
+    pos = torch.randint(C, w.max_pos + 1, (w.S,), generator=g, dtype=torch.int64)
+    return Q, K, V, pos.to(torch.int32).to(device)
+
+
+def window_slots_in_key_order(p: int, window: int, n_global: int):
+    """Cache slots of the index set of a query at position p, in ascending key
+    order (globals, then the window), for a cache of window + n_global slots."""
+    keys = np.concatenate([np.arange(min(n_global, p + 1)),
+                           np.arange(max(n_global, p - window + 1), p + 1)])
+    return np.where(keys < n_global, keys, n_global + keys % window).astype(np.int64)
 
 
 def gather_index_sets(S: int, H_idx: int, L: int, n_idx: int, n_recent: int, seed: int,

@@ -9,7 +9,7 @@
  *   softmax(Q K^T / sqrt(d_k)) V ("sparse attention mechanism" glossary,
  *   chipfoundryservices, "Standard Attention Bottleneck").
  *
- * G_i comes from one of two places:
+ * G_i comes from one of three places:
  *   - sparse_attn_prefill*: a static pattern (sa_pattern_t) -- the union, by
  *     logical OR ("SAS: Sparse Attention Synthesizer", kindchill, Step 5,
  *     component 2), of a sliding window, global tokens, block-local blocks and
@@ -21,7 +21,9 @@
  *     computed, its maximum scaled logit is compared with a per-head calibrated
  *     threshold, and below it the block's V load and PV product are skipped and
  *     its keys leave G_i for every row of the 128-row query tile.
- *   - sparse_attn_gather: explicit, sorted index sets over a KV cache (decode).
+ *   - sparse_attn_gather: explicit index sets over a KV cache (decode).
+ *   - sparse_attn_decode_window: the decode row of a causal window + global
+ *     tokens pattern, over a cache of window + globals slots.
  *
  * K/V heads are shared by contiguous groups of query heads (GQA/MQA, glossary
  * "Multi-Query and Grouped-Query Attention"): h_kv = h / (H / H_kv).
@@ -192,9 +194,10 @@ int sparse_attn_calibrate(const sa_plan_t *plan, const float *block_stat, double
 
 /* Explicit index-set attention over a KV cache (decode, one query per sequence).
  *   Q [S][H][d] bf16; K, V [S][H_kv][L][d] bf16; O [S][H][d] bf16 (written).
- *   idx: device int32 [S][H_idx][n_idx]; each set sorted ascending, unique, in
- *        [0, L).  H_idx == H: one set per query head; H_idx == H_kv: one set per
- *        K/V head, shared by its query heads.
+ *   idx: device int32 [S][H_idx][n_idx]; each set unique, in [0, L); rows are
+ *        visited in the order given (the workloads pass them sorted ascending;
+ *        the order changes only the rounding).  H_idx == H: one set per query
+ *        head; H_idx == H_kv: one set per K/V head, shared by its query heads.
  *   idx_len: device int32 [S][H_idx] (entries used, 0..n_idx) or NULL (= n_idx).
  *   lse_out: device float [S][H] or NULL.
  *   An empty set gives O = 0, lse = -inf.  An index outside [0, L) is skipped
@@ -203,6 +206,34 @@ int sparse_attn_gather(const void *Q, const void *K, const void *V, const int32_
                        const int32_t *idx_len, void *O, int S, int H, int H_kv, int H_idx,
                        int L, int n_idx, int d, float scale, float *lse_out,
                        sa_stream_t stream);
+
+/* Decode over a minimum-size KV cache for the causal pattern "sliding window
+ * of W keys OR the first g (global) tokens" (glossary, "Mistral/Mixtral
+ * Sliding Window Attention" and "Sparse Attention Patterns"; the cache that
+ * the SAS tutorial's geometric pattern analyzer sizes from the pattern, Step 5,
+ * component 3).  The query of sequence s sits at position p = positions[s]; its
+ * index set is G_p = [0, min(g, p+1)) u [max(g, p-W+1), p], derived on the
+ * device from the descriptor -- no index array.
+ *   pat: causal = 1, window = W >= 1, n_global = g >= 0; no block_local, no
+ *        random blocks, no thresholds (otherwise SA_ERR_UNSUPPORTED); scale as
+ *        in sa_pattern_t.
+ *   Cache: K, V [S][H_kv][C][d] bf16 with C = W + g slots per (sequence, K/V
+ *        head): key j lives in slot sparse_attn_window_slot(j, W, g) (j for
+ *        j < g, else g + (j mod W)); the caller writes keys 0..p in order, so
+ *        the ring slots hold the last W keys.
+ *   Q [S][H][d] bf16, O [S][H][d] bf16 (written), positions device int32 [S],
+ *   lse_out device float [S][H] or NULL.  Rows are visited in ascending key
+ *   order, so the result equals sparse_attn_gather over the same cache with
+ *   the slots of G_p as the index set.  A negative position is recorded as
+ *   SA_ERR_DEVICE_INDEX and gives O = 0, lse = -inf. */
+int sparse_attn_decode_window(const void *Q, const void *K, const void *V,
+                              const int32_t *positions, void *O, int S, int H, int H_kv,
+                              int d, const sa_pattern_t *pat, float *lse_out,
+                              sa_stream_t stream);
+
+/* Cache slot of key j (j >= 0) in the layout of sparse_attn_decode_window;
+ * -1 when j < 0, window < 1 or n_global < 0.  Host only. */
+int64_t sparse_attn_window_slot(int64_t j, int window, int n_global);
 
 /* Prefill that allocates no device memory.  (The pages have no counterpart:
  * this is a deployment variant of sparse_attn_prefill.)  For callers that

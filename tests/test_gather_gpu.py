@@ -18,9 +18,13 @@ def _rand(shape, seed, device):
 
 @pytest.mark.parametrize("d,H,Hkv,H_idx,L,n_idx", [
     (128, 8, 2, 8, 1000, 300),
-    (128, 8, 2, 2, 1000, 300),
+    (128, 8, 2, 2, 1000, 300),      # shared sets, 4 query heads per K/V head
+    (128, 4, 2, 2, 700, 129),       # shared sets, 2 per K/V head
+    (64, 8, 2, 2, 640, 200),
+    (64, 4, 2, 2, 333, 57),
     (64, 4, 4, 4, 517, 517),
     (64, 6, 1, 6, 300, 33),
+    (64, 6, 1, 1, 300, 33),         # shared sets, 6 per K/V head (one CTA per query head)
 ])
 def test_gather_small(product, oracle_mod, cuda, d, H, Hkv, H_idx, L, n_idx):
     S = 3
@@ -49,6 +53,25 @@ def test_gather_ragged_lengths(product, oracle_mod, cuda):
     assert_close(O, Or)
     assert_close(lse, lr, what="lse")
     assert torch.all(O[lens == 0] == 0)
+
+
+@pytest.mark.parametrize("d,H,Hkv", [(128, 8, 2), (64, 4, 2)])
+def test_gather_shared_sets_same_bytes_as_per_head_sets(product, cuda, d, H, Hkv):
+    """Sets shared by the query heads of a K/V head (one CTA reads each row once
+    for all of them) give the same bytes as the same sets given per query head."""
+    S, L, n_idx = 3, 800, 250
+    Q, K, V = _rand((S, H, d), 21, cuda), _rand((S, Hkv, L, d), 22, cuda), _rand((S, Hkv, L, d), 23, cuda)
+    idx = gather_index_sets(S, Hkv, L, n_idx, 16, seed=24).to(cuda)
+    lens = torch.randint(0, n_idx + 1, (S, Hkv), dtype=torch.int32,
+                         generator=torch.Generator().manual_seed(25)).to(cuda)
+    l1, l2 = torch.empty((S, H), device=cuda), torch.empty((S, H), device=cuda)
+    O1 = product.sparse_attn_gather(Q, K, V, idx, idx_len=lens, lse=l1)
+    per_head = idx.repeat_interleave(H // Hkv, dim=1).contiguous()
+    lens_h = lens.repeat_interleave(H // Hkv, dim=1).contiguous()
+    O2 = product.sparse_attn_gather(Q, K, V, per_head, idx_len=lens_h, lse=l2)
+    product.check_device_error()
+    assert torch.equal(O1, O2)
+    assert torch.equal(l1, l2)
 
 
 def test_gather_bad_index_is_reported(product, cuda):
