@@ -361,15 +361,20 @@ def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
     from block_sparse_attention_29_b200 import compile_pattern, Pattern
     row_ptr, kb, full, cnt, H_pat, T = compile_pattern(Pattern(**w.pattern_fields(),
                                                                random_table=tab), w.H, w.N)
+    # a dilated window's tiles are 128 positions of one residue class r:
+    # rows (t*128 + m)*k + r
+    k = max(1, w.dilation)
+    n_pos = w.N // k
     flops_done, t_total, tiles_done, n = 0, 0.0, 0, 1
     while t_total < seconds:
-        tiles = [(int(g.integers(w.B)), int(g.integers(w.H)), int(g.integers(T))) for _ in range(n)]
-        rows = np.array([(b, h, i) for b, h, t in tiles
-                         for i in range(t * 128, min(w.N, t * 128 + 128))], np.int32)
+        tiles = [(int(g.integers(w.B)), int(g.integers(w.H)), int(g.integers(T)),
+                  int(g.integers(k))) for _ in range(n)]
+        rows = np.array([(b, h, m * k + r) for b, h, t, r in tiles
+                         for m in range(t * 128, min(n_pos, t * 128 + 128))], np.int32)
         t0 = time.perf_counter()
         oracle.prefill(opat, Qh, Kh, Vh, thresholds=thresholds, rows=rows, nthreads=cores)
         t_total += time.perf_counter() - t0
-        for b, h, t in tiles:
+        for b, h, t, _r in tiles:
             hp = h if H_pat > 1 else 0
             nb = int(row_ptr[hp * T + t + 1] - row_ptr[hp * T + t])
             flops_done += 4 * 128 * 64 * w.d * nb
@@ -535,7 +540,7 @@ def config_of(w, world):
         return {"workload": w.name, "sequences": w.S, "H": w.H, "H_kv": w.H_kv, "d": w.d,
                 "cache_len": w.L, "n_idx": w.n_idx, "H_idx": w.H_idx,
                 "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}
-    pat = {k: v for k, v in w.pattern_fields().items() if v}
+    pat = {k: v for k, v in w.pattern_fields().items() if v and not (k == "dilation" and v == 1)}
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
             "pattern": pat, "block_skip_rule": bool(w.bsfa),
             "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}

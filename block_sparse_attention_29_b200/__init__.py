@@ -46,6 +46,7 @@ class Pattern:
     n_random: int = 0
     random_table: Optional[np.ndarray] = None   # host int32 [H][ceil(N/rb)][n_random]
     scale: float = 0.0
+    dilation: int = 1   # window taps this far apart (dilated/strided window); 1 = contiguous
 
     def to_c(self, thresholds_ptr: int = 0):
         tab = None
@@ -54,7 +55,7 @@ class Pattern:
         st = SaPattern(self.causal, self.window, self.n_global, self.block_local, self.block_q,
                        self.block_k, self.random_block, self.n_random if tab is not None else 0,
                        tab.ctypes.data if tab is not None else None,
-                       thresholds_ptr or None, self.scale)
+                       thresholds_ptr or None, self.scale, self.dilation)
         return st, tab   # the caller keeps `tab` alive while the struct is used
 
 

@@ -90,16 +90,22 @@ int check_current_device(int want) {
 }
 }  // namespace
 
-// 3-D bf16 map over a [BH][N][d] tensor, box {64, rows, 1}, 128-byte swizzle.
-// Rows past N read as zero.
-int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows) {
+// 4-D bf16 map over a [BH][N][d] tensor seen as [BH][N/dil][dil][d]:
+// coordinates (x, residue r, position m within the residue class, slice) address
+// row m*dil + r; box {64, 1, rows, 1}, 128-byte swizzle, so a box is `rows`
+// rows of one class, dil rows apart (dil = 1: plain consecutive rows).  Rows
+// past N/dil read as zero.  N % dil == 0 is checked by the caller, so no
+// in-bounds coordinate reaches past row N - 1 of its slice.
+int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows, int dil) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return set_error(SA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
-  const cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(N) * d * 2};
-  const cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  if (dil < 1 || N % dil != 0) return set_error(SA_ERR_INVALID_ARG, "dilation %d, N = %d", dil, N);
+  const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(dil), cuuint64_t(N / dil), cuuint64_t(BH)};
+  const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(dil) * d * 2,
+                                 cuuint64_t(N) * d * 2};
+  const cuuint32_t box[4] = {64, 1, cuuint32_t(rows), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
@@ -113,6 +119,7 @@ struct sa_plan {
   sa_pattern_t pat{};
   int B = 0, H = 0, Hkv = 0, N = 0, d = 0, device = 0;
   int T = 0, n_kb = 0, H_pat = 0;
+  int dil = 1;                 // dilation: the plan's lists cover one of dil residue classes
   int n_units = 0;
   bool pair = false;           // paired-head kernel (units are head pairs)
   int32_t* d_row_ptr = nullptr;
@@ -169,7 +176,8 @@ int check_shapes(const sa_pattern_t* pat, int B, int H, int Hkv, int N, int d) {
     return set_error(SA_ERR_UNSUPPORTED, "random_block = %d must be a positive multiple of 64",
                      pat->random_block);
   if (N >= (1 << 28)) return set_error(SA_ERR_UNSUPPORTED, "N = %d too large", N);
-  const int64_t units = int64_t(B) * H * ((N + kTileQ - 1) / kTileQ);
+  const int dil = pat->dilation > 1 ? pat->dilation : 1;
+  const int64_t units = int64_t(B) * dil * H * ((N / dil + kTileQ - 1) / kTileQ);
   if (units > INT32_MAX) return set_error(SA_ERR_UNSUPPORTED, "B*H*tiles too large");
   if (int64_t(B) * H > 65535 || int64_t(B) * Hkv > 65535)
     return set_error(SA_ERR_UNSUPPORTED, "B*H must not exceed 65535");
@@ -182,7 +190,8 @@ std::string cache_key(const sa_pattern_t* p, int B, int H, int Hkv, int N, int d
   std::string k;
   auto put = [&k](const void* src, size_t n) { k.append(static_cast<const char*>(src), n); };
   const int32_t f[] = {p->causal, p->window, p->n_global, p->block_local, p->block_q,
-                       p->block_k, p->random_block, p->n_random, B, H, Hkv, N, d, dev};
+                       p->block_k, p->random_block, p->n_random, p->dilation > 1 ? p->dilation : 1,
+                       B, H, Hkv, N, d, dev};
   put(f, sizeof f);
   put(&p->scale, sizeof p->scale);
   if (p->n_random > 0 && p->random_table && p->random_block > 0) {
@@ -202,9 +211,10 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
                         void* O, const float* thresholds, float* lse, uint8_t* mask,
                         float* stat, PrefillParams* p) {
   std::memset(p, 0, sizeof *p);
-  int rc = make_tmap(&p->tm_q, Q, plan->d, plan->N, plan->B * plan->H, kTileQ);
-  if (!rc) rc = make_tmap(&p->tm_k, K, plan->d, plan->N, plan->B * plan->Hkv, kTileK);
-  if (!rc) rc = make_tmap(&p->tm_v, V, plan->d, plan->N, plan->B * plan->Hkv, kTileK);
+  const int dil = plan->dil;
+  int rc = make_tmap(&p->tm_q, Q, plan->d, plan->N, plan->B * plan->H, kTileQ, dil);
+  if (!rc) rc = make_tmap(&p->tm_k, K, plan->d, plan->N, plan->B * plan->Hkv, kTileK, dil);
+  if (!rc) rc = make_tmap(&p->tm_v, V, plan->d, plan->N, plan->B * plan->Hkv, kTileK, dil);
   if (rc) return rc;
   p->O = static_cast<uint16_t*>(O);
   p->lse = lse;
@@ -221,7 +231,8 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
   p->B = plan->B;
   p->H = plan->H;
   p->Hkv = plan->Hkv;
-  p->N = plan->N;
+  p->N = plan->N / dil;
+  p->dil = dil;
   p->T = plan->T;
   p->n_kb = plan->n_kb;
   p->head_pat = plan->H_pat > 1 ? 1 : 0;
@@ -282,10 +293,11 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
   CompiledPattern cp;
   rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
   if (rc) return rc;
-  if (kernel == SA_KERNEL_PAIRED_HEADS && !pair_kernel_fits(d, H, H_kv, cp.H_pat))
+  const int dil = pat->dilation > 1 ? pat->dilation : 1;
+  if (kernel == SA_KERNEL_PAIRED_HEADS && (dil > 1 || !pair_kernel_fits(d, H, H_kv, cp.H_pat)))
     return set_error(SA_ERR_UNSUPPORTED,
                      "the paired-head kernel needs d = 128, an even number of query heads per "
-                     "K/V head and no random table");
+                     "K/V head, no random table and no dilation");
 
   sa_plan_t* plan = new sa_plan_t;
   plan->pat = *pat;
@@ -299,6 +311,7 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
   plan->T = cp.T;
   plan->n_kb = cp.n_kb;
   plan->H_pat = cp.H_pat;
+  plan->dil = dil;
   cudaGetDevice(&plan->device);
 
   // Block lists as packed entries; accounting over all (b, h).
@@ -310,10 +323,12 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
     per_pat_pairs += cp.cnt[e];
   }
   per_pat_blocks = int64_t(cp.kb.size());
-  const int64_t rep = int64_t(B) * (cp.H_pat == 1 ? H : 1);
+  // B*dil independent sequences: each residue class of a dilated window runs the lists
+  const int Bd = B * dil;
+  const int64_t rep = int64_t(Bd) * (cp.H_pat == 1 ? H : 1);
   plan->info.T_q = cp.T;
   plan->info.n_kb = cp.n_kb;
-  plan->info.n_units = int64_t(B) * H * cp.T;
+  plan->info.n_units = int64_t(Bd) * H * cp.T;
   plan->info.blocks = per_pat_blocks * rep;
   plan->info.blocks_full = per_pat_full * rep;
   plan->info.pairs = per_pat_pairs * rep;
@@ -326,14 +341,14 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
       delete plan;
       return rc;
     }
-    plan->info.blocks_desc = int64_t(cd.kb.size()) * int64_t(B) * (cd.H_pat == 1 ? H : 1);
+    plan->info.blocks_desc = int64_t(cd.kb.size()) * int64_t(Bd) * (cd.H_pat == 1 ? H : 1);
   }
 
   plan->pair = kernel == SA_KERNEL_PAIRED_HEADS;
   plan->info.paired_heads = plan->pair ? 1 : 0;
-  plan->n_units = B * cp.T * (plan->pair ? H / 2 : H);
+  plan->n_units = Bd * cp.T * (plan->pair ? H / 2 : H);
   std::vector<int32_t> units;
-  build_units(cp, B, H, H_kv, N, d, plan->pair, &units);
+  build_units(cp, Bd, H, H_kv, N / dil, d, plan->pair, &units);
 
   rc = upload(&plan->d_row_ptr, cp.row_ptr.data(), cp.row_ptr.size());
   if (!rc) rc = upload(&plan->d_entries, entries.data(), entries.size());
@@ -373,6 +388,9 @@ int sparse_attn_prefill_plan(const sa_plan_t* plan, const void* Q, const void* K
     return set_error(SA_ERR_INVALID_ARG, "Q, K, V and O must be 16-byte aligned");
   if (thresholds && plan->pat.block_q != kTileQ)
     return set_error(SA_ERR_UNSUPPORTED, "the block-skip rule needs block_q = 128");
+  if (plan->dil > 1 && (thresholds || block_mask_out || block_stat_out))
+    return set_error(SA_ERR_UNSUPPORTED,
+                     "a dilated plan takes no thresholds, block mask or block statistics");
   int rc = check_current_device(plan->device);
   if (rc) return rc;
   PrefillParams p;
@@ -398,6 +416,7 @@ int sparse_attn_block_stats(const sa_plan_t* plan, const void* Q, const void* K,
   if (!aligned16(Q) || !aligned16(K)) return set_error(SA_ERR_INVALID_ARG, "Q and K must be 16-byte aligned");
   if (plan->pat.block_q != kTileQ)
     return set_error(SA_ERR_UNSUPPORTED, "the block-skip rule needs block_q = 128");
+  if (plan->dil > 1) return set_error(SA_ERR_UNSUPPORTED, "no block statistics for a dilated plan");
   int rc = check_current_device(plan->device);
   if (rc) return rc;
   PrefillParams p;
@@ -422,6 +441,7 @@ int sparse_attn_calibrate(const sa_plan_t* plan, const float* block_stat, double
   if (!plan || !block_stat || !thresholds_out)
     return set_error(SA_ERR_INVALID_ARG, "plan, block_stat and thresholds_out must be non-NULL");
   if (!(q >= 0.0 && q <= 1.0)) return set_error(SA_ERR_INVALID_ARG, "q = %g outside [0, 1]", q);
+  if (plan->dil > 1) return set_error(SA_ERR_UNSUPPORTED, "no calibration for a dilated plan");
   int rc = check_current_device(plan->device);
   if (rc) return rc;
   return launch_calibrate(block_stat, plan->d_row_ptr, plan->d_entries, plan->H_pat > 1 ? 1 : 0,
@@ -508,10 +528,11 @@ int sparse_attn_decode_window(const void* Q, const void* K, const void* V,
   if (!pat->causal || pat->window < 1 || pat->n_global < 0)
     return set_error(SA_ERR_UNSUPPORTED,
                      "window decode needs a causal pattern with window >= 1 and n_global >= 0");
-  if (pat->block_local > 0 || (pat->n_random > 0 && pat->random_table) || pat->thresholds)
+  if (pat->block_local > 0 || (pat->n_random > 0 && pat->random_table) || pat->thresholds ||
+      pat->dilation > 1)
     return set_error(SA_ERR_UNSUPPORTED,
                      "window decode covers the window and global tokens only (no block_local, "
-                     "random blocks or thresholds)");
+                     "random blocks, dilation or thresholds)");
   const int64_t C = int64_t(pat->window) + pat->n_global;
   if (C > INT32_MAX) return set_error(SA_ERR_UNSUPPORTED, "cache of %lld slots too large", (long long)C);
   GatherParams p;

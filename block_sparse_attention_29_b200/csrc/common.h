@@ -35,8 +35,8 @@ __host__ __device__ inline int32_t entry_pack(int32_t kb, bool partial) {
 }
 
 struct PrefillParams {
-  CUtensorMap tm_q;   // 3-D {d, N, B*H}    box {64, 128, 1}, 128-B swizzle
-  CUtensorMap tm_k;   // 3-D {d, N, B*H_kv} box {64, 64, 1},  128-B swizzle
+  CUtensorMap tm_q;   // 4-D {d, dil, N/dil, B*H}    box {64, 1, 128, 1}, 128-B swizzle
+  CUtensorMap tm_k;   // 4-D {d, dil, N/dil, B*H_kv} box {64, 1, 64, 1},  128-B swizzle
   CUtensorMap tm_v;   // same as tm_k over V
   uint16_t* O;        // [B][H][N][d] bf16
   float* lse;         // [B][H][N] or null
@@ -44,14 +44,17 @@ struct PrefillParams {
   float* stat_out;    // [B][H][T][n_kb] or null
   const int32_t* row_ptr;   // [H_pat*T + 1]
   const int32_t* entries;   // block lists
-  const int32_t* units;     // work order: unit = (b*H + h)*T + t, or with pair = 1
-                            // (b*(H/2) + hp)*T + t for the heads 2hp and 2hp + 1
+  const int32_t* units;     // work order: unit = (b'*H + h)*T + t, or with pair = 1
+                            // (b'*(H/2) + hp)*T + t for the heads 2hp and 2hp + 1;
+                            // b' = b*dil + residue class (b' = b without dilation)
   int* sched;               // [2] work-queue counters (next unit, CTAs done); zero
                             // between launches (the last CTA of a launch resets them)
   const int32_t* rtab;      // random table [H][n_rb][n_random] or null
   const float* thresholds;  // [H] or null
   int n_units;
-  int B, H, Hkv, N, T, n_kb, head_pat;   // head_pat: 1 when lists are per head
+  int B, H, Hkv, N, T, n_kb, head_pat;   // head_pat: 1 when lists are per head;
+                                         // N: positions per residue class (N/dil)
+  int dil;         // dilation: query/key position m of class r is row m*dil + r
   int causal, window, n_global, block_local, random_block, n_random;
   int pair;        // 1: units are head pairs (paired-head kernel), 0: single heads
   int gate;        // 1: statistics + decision per block (rule or stats pass)
@@ -73,9 +76,10 @@ inline bool pair_kernel_fits(int d, int H, int H_kv, int H_pat) {
   return d == 128 && H_pat == 1 && H % H_kv == 0 && (H / H_kv) % 2 == 0;
 }
 
-// 3-D bf16 TMA map over a [BH][N][d] tensor, box {64, rows, 1}, 128-byte
-// swizzle; rows past N read as zero.
-int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows);
+// 4-D bf16 TMA map over a [BH][N][d] tensor seen as [BH][N/dil][dil][d]:
+// coordinates (x, r, m, slice) address row m*dil + r; box {64, 1, rows, 1},
+// 128-byte swizzle; positions m past N/dil read as zero.  N % dil == 0.
+int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows, int dil);
 
 // ----------------------------------------------------------------- gather --
 struct GatherParams {

@@ -93,7 +93,10 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   if (rc) return rc;
   const int T = cp.T;
   const bool pair = false;   // the single-head kernel (the default of the plan API)
-  const int64_t n_units = int64_t(B) * (pair ? H / 2 : H) * T;
+  const int dil = pat->dilation > 1 ? pat->dilation : 1;
+  if (dil > 1 && pat->thresholds)
+    return set_error(SA_ERR_UNSUPPORTED, "a dilated window takes no block-skip thresholds");
+  const int64_t n_units = int64_t(B) * dil * (pair ? H / 2 : H) * T;
   const int nrb = rnd ? (N + pat->random_block - 1) / pat->random_block : 0;
   const size_t b_row = round256(cp.row_ptr.size() * 4);
   const size_t b_ent = round256(std::max<size_t>(cp.kb.size(), 1) * 4);
@@ -110,7 +113,7 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   std::vector<int32_t> entries(cp.kb.size());
   for (size_t e = 0; e < cp.kb.size(); ++e) entries[e] = entry_pack(cp.kb[e], !cp.full[e]);
   std::vector<int32_t> units;
-  build_units(cp, B, H, H_kv, N, d, pair, &units);
+  build_units(cp, B * dil, H, H_kv, N / dil, d, pair, &units);
 
   unsigned char* base = nullptr;
   rc = scratch_address(&base);
@@ -139,9 +142,9 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
 
   PrefillParams p;
   std::memset(&p, 0, sizeof p);
-  rc = make_tmap(&p.tm_q, Q, d, N, B * H, kTileQ);
-  if (!rc) rc = make_tmap(&p.tm_k, K, d, N, B * H_kv, kTileK);
-  if (!rc) rc = make_tmap(&p.tm_v, V, d, N, B * H_kv, kTileK);
+  rc = make_tmap(&p.tm_q, Q, d, N, B * H, kTileQ, dil);
+  if (!rc) rc = make_tmap(&p.tm_k, K, d, N, B * H_kv, kTileK, dil);
+  if (!rc) rc = make_tmap(&p.tm_v, V, d, N, B * H_kv, kTileK, dil);
   if (rc) return rc;
   p.O = static_cast<uint16_t*>(O);
   p.lse = lse_out;
@@ -156,7 +159,8 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   p.B = B;
   p.H = H;
   p.Hkv = H_kv;
-  p.N = N;
+  p.N = N / dil;
+  p.dil = dil;
   p.T = T;
   p.n_kb = cp.n_kb;
   p.head_pat = cp.H_pat > 1 ? 1 : 0;

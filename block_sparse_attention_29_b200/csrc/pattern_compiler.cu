@@ -12,6 +12,13 @@
 // the two edge blocks get their partial lengths.  A block is listed when it
 // holds at least one visible pair and is "full" when it holds tile_q*tile_k
 // (every pair of the tile, which also rules out ragged tiles and blocks).
+//
+// A dilated window (dilation k > 1: taps k apart, glossary "Sparse Attention
+// Patterns", dilated/strided row) only joins i and j of one residue class
+// i mod k, and inside a class, numbered m = i / k, it is the contiguous window
+// over N/k positions.  The compiler therefore lists the contiguous window over
+// N/k positions once; the kernels run it for every class through a strided
+// view of Q, K, V and O.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
@@ -70,6 +77,17 @@ int validate_pattern(const sa_pattern_t* p, int H, int N) {
     return set_error(SA_ERR_INVALID_ARG, "negative pattern field");
   if (p->block_q <= 0 || p->block_k <= 0)
     return set_error(SA_ERR_INVALID_ARG, "block_q and block_k must be positive");
+  if (p->dilation < 0) return set_error(SA_ERR_INVALID_ARG, "negative dilation");
+  if (p->dilation > 1) {
+    if (p->window <= 0)
+      return set_error(SA_ERR_INVALID_ARG, "dilation %d needs a window", p->dilation);
+    if (p->n_global > 0 || p->block_local > 0 || (p->n_random > 0 && p->random_table))
+      return set_error(SA_ERR_UNSUPPORTED,
+                       "a dilated window cannot be combined with other primitives");
+    if (N % p->dilation != 0)
+      return set_error(SA_ERR_UNSUPPORTED, "dilation %d does not divide N = %d", p->dilation,
+                       N);
+  }
   if (p->n_random > 0 && p->random_table != nullptr) {
     if (p->random_block <= 0)
       return set_error(SA_ERR_INVALID_ARG, "random_block must be positive");
@@ -89,6 +107,11 @@ int compile_pattern(const sa_pattern_t* p, int H, int N, int tile_q, int tile_k,
                     CompiledPattern* out) {
   int rc = validate_pattern(p, H, N);
   if (rc) return rc;
+  if (p->dilation > 1) {   // one residue class: the contiguous window over N/k positions
+    sa_pattern_t c = *p;
+    c.dilation = 1;
+    return compile_pattern(&c, H, N / p->dilation, tile_q, tile_k, out);
+  }
   if (tile_q <= 0 || tile_k <= 0) return set_error(SA_ERR_INVALID_ARG, "bad tile size");
   const int H_pat = random_on(p) ? H : 1;
   const int T = (N + tile_q - 1) / tile_q;

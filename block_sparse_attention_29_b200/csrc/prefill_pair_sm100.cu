@@ -192,8 +192,8 @@ __device__ void producer2(const PrefillParams& p, uint8_t* smem, Bars2* bars) {
     mbar_expect_tx(smem_u32(&bars->q_full), 2 * Q_BYTES);
     for (int x = 0; x < 2; ++x)
       for (int c = 0; c < 2; ++c)
-        tma_load_3d(sQ + x * Q_BYTES + c * (kTileQ * 128), &p.tm_q, smem_u32(&bars->q_full),
-                    c * 64, u.t * kTileQ, u.b * p.H + 2 * u.hp + x);
+        tma_load_4d(sQ + x * Q_BYTES + c * (kTileQ * 128), &p.tm_q, smem_u32(&bars->q_full),
+                    c * 64, 0, u.t * kTileQ, u.b * p.H + 2 * u.hp + x);
     ++qc;
     for (int j = 0; j < u.n; j += 2) {
       const int nb = min(2, u.n - j);
@@ -206,8 +206,8 @@ __device__ void producer2(const PrefillParams& p, uint8_t* smem, Bars2* bars) {
       for (int hb = 0; hb < nb; ++hb) {
         const int kb = __ldg(p.entries + u.beg + j + hb) >> 1;
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(dst + c * (2 * kTileK * 128) + hb * (kTileK * 128), &p.tm_k,
-                      smem_u32(&bars->k_full[st]), c * 64, kb * kTileK, u.b * p.Hkv + u.hkv);
+          tma_load_4d(dst + c * (2 * kTileK * 128) + hb * (kTileK * 128), &p.tm_k,
+                      smem_u32(&bars->k_full[st]), c * 64, 0, kb * kTileK, u.b * p.Hkv + u.hkv);
       }
       ++kc;
     }
@@ -232,7 +232,7 @@ __device__ __forceinline__ void load_v_half(const PrefillParams& p, Bars2* bars,
   const uint32_t bar = smem_u32(&bars->v_full[st][hb]);
   mbar_expect_tx(bar, HALF_BYTES);
   for (int c = 0; c < 2; ++c)
-    tma_load_3d(base + hb * HALF_BYTES + c * (kTileK * 128), &p.tm_v, bar, c * 64, kb * kTileK,
+    tma_load_4d(base + hb * HALF_BYTES + c * (kTileK * 128), &p.tm_v, bar, c * 64, 0, kb * kTileK,
                 u.b * p.Hkv + u.hkv);
 }
 
@@ -771,6 +771,7 @@ int launch_prefill_pair(const PrefillParams& p, int d, cudaStream_t stream) {
   if (d != kD) return set_error(SA_ERR_UNSUPPORTED, "paired-head kernel: head dim %d", d);
   if (p.head_pat || p.H % 2 || (p.H / p.Hkv) % 2)
     return set_error(SA_ERR_INVALID_ARG, "paired-head kernel: heads cannot be paired");
+  if (p.dil != 1) return set_error(SA_ERR_UNSUPPORTED, "paired-head kernel: dilated window");
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");

@@ -80,7 +80,7 @@ struct Cfg {
 };
 
 struct Unit {
-  int b, h, hkv, t, beg, n;
+  int b, r, h, hkv, t, beg, n;   // r: residue class of a dilated window (0 otherwise)
 };
 
 struct Bars {
@@ -109,7 +109,9 @@ __device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
   u.t = id % p.T;
   const int bh = id / p.T;
   u.h = bh % p.H;
-  u.b = bh / p.H;
+  const int bd = bh / p.H;   // b*dil + r
+  u.b = bd / p.dil;
+  u.r = bd - u.b * p.dil;
   u.hkv = u.h / (p.H / p.Hkv);
   const int row = (p.head_pat ? u.h : 0) * p.T + u.t;
   u.beg = __ldg(p.row_ptr + row);
@@ -134,11 +136,11 @@ __device__ __forceinline__ bool publish_unit(const PrefillParams& p, Bars* bars,
   if (v < p.n_units) {
     u = get_unit(p, v);
   } else {
-    u.b = u.h = u.hkv = u.t = u.beg = 0;
+    u.b = u.r = u.h = u.hkv = u.t = u.beg = 0;
     u.n = -1;
   }
   volatile int* d = reinterpret_cast<volatile int*>(&bars->unit_slot[slot]);
-  d[0] = u.b; d[1] = u.h; d[2] = u.hkv; d[3] = u.t; d[4] = u.beg; d[5] = u.n;
+  d[0] = u.b; d[1] = u.h; d[2] = u.hkv; d[3] = u.t; d[4] = u.beg; d[5] = u.n; d[6] = u.r;
   mbar_arrive(smem_u32(&bars->u_full[slot]));
   *out = u;
   return true;
@@ -155,6 +157,7 @@ __device__ __forceinline__ bool take_unit(const PrefillParams& p, Bars* bars, ui
     return false;
   const volatile int* d = reinterpret_cast<const volatile int*>(&bars->unit_slot[slot]);
   out->b = d[0]; out->h = d[1]; out->hkv = d[2]; out->t = d[3]; out->beg = d[4]; out->n = d[5];
+  out->r = d[6];
   if (whole_warp) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&bars->u_empty[slot]));
@@ -181,7 +184,7 @@ __device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars)
       goto drain;
     mbar_expect_tx(smem_u32(&bars->q_full), C::Q_BYTES);
     for (int c = 0; c < C::CH; ++c)
-      tma_load_3d(sQ + c * (kTileQ * 128), &p.tm_q, smem_u32(&bars->q_full), c * 64,
+      tma_load_4d(sQ + c * (kTileQ * 128), &p.tm_q, smem_u32(&bars->q_full), c * 64, u.r,
                   u.t * kTileQ, u.b * p.H + u.h);
     ++qc;
     for (int k = 0; k < u.n; ++k) {
@@ -193,8 +196,8 @@ __device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars)
       const uint32_t dst = sK + st * C::KV_BYTES;
       mbar_expect_tx(smem_u32(&bars->k_full[st]), C::KV_BYTES);
       for (int c = 0; c < C::CH; ++c)
-        tma_load_3d(dst + c * (kTileK * 128), &p.tm_k, smem_u32(&bars->k_full[st]), c * 64,
-                    kb * kTileK, u.b * p.Hkv + u.hkv);
+        tma_load_4d(dst + c * (kTileK * 128), &p.tm_k, smem_u32(&bars->k_full[st]), c * 64,
+                    u.r, kb * kTileK, u.b * p.Hkv + u.hkv);
       ++kc;
     }
   }
@@ -241,8 +244,8 @@ __device__ void vloader_role(const PrefillParams& p, uint8_t* smem, Bars* bars) 
       const uint32_t dst = sV + vs * C::KV_BYTES;
       mbar_expect_tx(smem_u32(&bars->v_full[vs]), C::KV_BYTES);
       for (int c = 0; c < C::CH; ++c)
-        tma_load_3d(dst + c * (kTileK * 128), &p.tm_v, smem_u32(&bars->v_full[vs]), c * 64,
-                    kb * kTileK, u.b * p.Hkv + u.hkv);
+        tma_load_4d(dst + c * (kTileK * 128), &p.tm_v, smem_u32(&bars->v_full[vs]), c * 64,
+                    u.r, kb * kTileK, u.b * p.Hkv + u.hkv);
       ++vc;
     }
   }
@@ -401,7 +404,8 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
     if (u.n < 0) break;
     const int i = u.t * kTileQ + row;
     const bool row_ok = i < p.N;
-    const int64_t orow = ((int64_t)(u.b * p.H + u.h) * p.N + i);
+    // output row: position i of residue class u.r is row i*dil + r of the slice
+    const int64_t orow = (int64_t)(u.b * p.H + u.h) * p.N * p.dil + (int64_t)i * p.dil + u.r;
     const int64_t tile_base = ((int64_t)(u.b * p.H + u.h) * p.T + u.t) * p.n_kb;
     const float tau = (p.gate && !p.stats_only) ? __ldg(p.thresholds + u.h) : 0.f;
     float m = -INFINITY, l = 0.f;

@@ -19,6 +19,10 @@ Workloads (names used by tests and bench):
   gather_decode       64 sequences x 1 query, H=32 H_kv=8 d=128, cache length 131072,
                       2048 sorted unique indices per (sequence, head) = {0} and the last
                       128 positions and 1919 uniform draws from {1 .. L-129}
+  window_decode       64 sequences x 1 query, H=32 H_kv=8 d=128, causal window 4096 +
+                      4 global tokens over a cache of 4100 slots, positions past the window
+  dilated_swa         B=1 H=32 H_kv=8 N=32768 d=128, causal dilated window: 2048 taps
+                      8 apart (receptive field 16384), blocks 128x64
 """
 from __future__ import annotations
 
@@ -47,12 +51,14 @@ class PrefillWorkload:
     n_random: int = 0
     bsfa: bool = False
     seed: int = 0
+    dilation: int = 1
     extra: dict = field(default_factory=dict)
 
     def pattern_fields(self):
         return dict(causal=self.causal, window=self.window, n_global=self.n_global,
                     block_local=self.block_local, block_q=self.block_q, block_k=self.block_k,
-                    random_block=self.random_block, n_random=self.n_random)
+                    random_block=self.random_block, n_random=self.n_random,
+                    dilation=self.dilation)
 
 
 @dataclass
@@ -99,6 +105,8 @@ WORKLOADS = {
                                     n_idx=2048, H_idx=32, seed=5000),
     "window_decode": WindowDecodeWorkload("window_decode", S=64, H=32, H_kv=8, d=128,
                                           window=4096, n_global=4, max_pos=131071, seed=6000),
+    "dilated_swa": PrefillWorkload("dilated_swa", B=1, H=32, H_kv=8, N=32768, d=128, causal=1,
+                                   window=2048, dilation=8, block_q=128, block_k=64, seed=7000),
 }
 
 

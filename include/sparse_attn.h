@@ -76,6 +76,15 @@ enum {
  *   random       n_random > 0 and random_table != NULL: key j is visible from
  *                query i when j / random_block is listed in
  *                random_table[h][i / random_block][0 .. n_random) (BigBird).
+ *   dilation     k > 1 makes the window dilated/strided (glossary "Sparse
+ *                Attention Patterns": attend to every k-th token, O(N*w)):
+ *                W taps k apart, i.e. (i - j) mod k == 0 and, with
+ *                m = (i - j) / k, 0 <= m < W (causal) or |m| <= W/2.  The kernels
+ *                run it as k independent sliding-window attentions, one per
+ *                residue class i mod k, read through a strided TMA view, so no
+ *                masked-out pair is computed.  Needs window > 0, no other
+ *                primitive, no block-skip thresholds and N % k == 0
+ *                (SA_ERR_UNSUPPORTED otherwise).  0 and 1 mean contiguous.
  * block_q x block_k is the tile of the block-skip rule and of the block FLOP
  * accounting.  The kernels tile 128 query rows x 64 keys, so block_k must be 64
  * and block_q 64 or 128 (128 when the block-skip rule is used).
@@ -98,6 +107,7 @@ typedef struct {
                                       Used by sparse_attn_prefill only; plans take the
                                       thresholds per call.                                */
     float scale;
+    int32_t dilation;              /* window taps k apart; 0 or 1 = contiguous window    */
 } sa_pattern_t;
 
 /* A compiled pattern: per-(head, 128-row query tile) lists of 64-key blocks
@@ -106,9 +116,10 @@ typedef struct {
 typedef struct sa_plan sa_plan_t;
 
 typedef struct {
-    int32_t T_q;            /* 128-row query tiles per (b, h): ceil(N/128)              */
-    int32_t n_kb;           /* 64-key blocks per row: ceil(N/64)                         */
-    int64_t n_units;        /* work units B*H*T_q                                        */
+    int32_t T_q;            /* 128-row query tiles per (b, h): ceil(N/128); with
+                               dilation k > 1, per (b, h, residue): ceil(N/k/128)       */
+    int32_t n_kb;           /* 64-key blocks per row: ceil(N/64) (ceil(N/k/64))          */
+    int64_t n_units;        /* work units B*H*T_q (B*k*H*T_q with dilation k > 1)        */
     int64_t blocks;         /* listed (tile, key block) pairs over all (b, h), 128x64   */
     int64_t blocks_full;    /* ... of which every pair is in G (may be skipped)         */
     int64_t blocks_desc;    /* listed blocks at the descriptor's block_q x block_k      */
@@ -133,8 +144,11 @@ enum {
 /* Compile `pat` for Q [B][H][N][d], K/V [B][H_kv][N][d].  Host work plus
  * cudaMalloc/cudaMemcpy on the current device; synchronous.  Errors:
  * SA_ERR_INVALID_ARG (shapes, H % H_kv != 0, bad descriptor or table entry),
- * SA_ERR_UNSUPPORTED (d not 64/128, block_k != 64, random_block % 64 != 0),
- * SA_ERR_NO_MEMORY, SA_ERR_CUDA.  On success *out owns the plan. */
+ * SA_ERR_UNSUPPORTED (d not 64/128, block_k != 64, random_block % 64 != 0,
+ * dilation k > 1 with another primitive or N % k != 0), SA_ERR_NO_MEMORY,
+ * SA_ERR_CUDA.  On success *out owns the plan.  A dilated plan (k > 1) holds
+ * the lists of the contiguous window over one residue class (N/k positions),
+ * shared by the k classes. */
 int sparse_attn_plan_create(const sa_pattern_t *pat, int B, int H, int H_kv, int N, int d,
                             sa_plan_t **out);
 /* Same as sparse_attn_plan_create with an explicit kernel choice (SA_KERNEL_*;
@@ -158,6 +172,8 @@ void sparse_attn_plan_destroy(sa_plan_t *plan);   /* synchronises the device; NU
  *   block_stat_out: device float [B][H][T_q][n_kb]; for listed blocks the
  *            maximum scaled logit over the tile's visible pairs (unlisted
  *            entries are left untouched); or NULL.
+ * A dilated plan takes no thresholds, block_mask_out or block_stat_out
+ * (SA_ERR_UNSUPPORTED): the block-skip rule is defined on contiguous tiles.
  * The plan must not be destroyed while a launch that uses it may still run,
  * and launches that use one plan must not overlap on the GPU (issue them on
  * one stream, or order them): the plan holds the launch's work-queue
@@ -178,7 +194,8 @@ int sparse_attn_prefill(const void *Q, const void *K, const void *V, void *O,
 /* Block-statistics pass of the block-skip rule over a plan: computes the
  * QK^T tiles of every listed block and writes block_stat_out (layout as
  * above) and block_mask_out (1 for every listed block); no V is read and no
- * output is written.  Used to calibrate thresholds on a calibration draw. */
+ * output is written.  Used to calibrate thresholds on a calibration draw.
+ * Dilated plans: SA_ERR_UNSUPPORTED. */
 int sparse_attn_block_stats(const sa_plan_t *plan, const void *Q, const void *K,
                             float *block_stat_out, uint8_t *block_mask_out,
                             sa_stream_t stream);
@@ -258,7 +275,9 @@ int sparse_attn_prefill_noalloc(const void *Q, const void *K, const void *V, voi
  * (the lists do not depend on the head).  First call with row_ptr == NULL to
  * get *H_pat_out, *T_out, *n_entries_out; then call again with
  * row_ptr int32 [H_pat*T + 1], kb int32 [n_entries], full uint8 [n_entries]
- * and, optionally, cnt int64 [n_entries] (visible pairs per listed block). */
+ * and, optionally, cnt int64 [n_entries] (visible pairs per listed block).
+ * With dilation k > 1 the lists are those of one residue class: the
+ * contiguous window over N/k positions (T = ceil(N/k/tile_q)). */
 int sparse_attn_compile_pattern(const sa_pattern_t *pat, int H, int N, int tile_q,
                                 int tile_k, int *H_pat_out, int *T_out,
                                 int64_t *n_entries_out, int32_t *row_ptr, int32_t *kb,

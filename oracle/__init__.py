@@ -59,7 +59,7 @@ class _Pattern(ctypes.Structure):
                 ("n_global", ctypes.c_int32), ("block_local", ctypes.c_int32),
                 ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
                 ("random_block", ctypes.c_int32), ("n_random", ctypes.c_int32),
-                ("random_table", ctypes.c_void_p)]
+                ("random_table", ctypes.c_void_p), ("dilation", ctypes.c_int32)]
 
 
 def _load():
@@ -101,6 +101,7 @@ class Pattern:
     random_block: int = 64
     n_random: int = 0
     random_table: Optional[np.ndarray] = None   # int32 [H][ceil(N/rb)][n_random]
+    dilation: int = 1   # window taps k apart (glossary table, dilated/strided row)
 
     def _c(self):
         tab = None
@@ -109,7 +110,7 @@ class Pattern:
         st = _Pattern(self.causal, self.window, self.n_global, self.block_local,
                       self.block_q, self.block_k, self.random_block,
                       self.n_random if tab is not None else 0,
-                      tab.ctypes.data if tab is not None else None)
+                      tab.ctypes.data if tab is not None else None, self.dilation)
         return st, tab          # keep tab alive alongside the struct
 
 
@@ -160,7 +161,12 @@ def visible_py(p: Pattern, N: int, h: int, i: int, j: int) -> bool:
         return False
     prims = []
     if p.window > 0:
-        prims.append((i - p.window < j <= i) if p.causal else (abs(i - j) <= p.window // 2))
+        k = max(1, p.dilation)
+        if (i - j) % k:
+            prims.append(False)       # not one of the window's taps
+        else:
+            m = (i - j) // k
+            prims.append((0 <= m < p.window) if p.causal else (abs(m) <= p.window // 2))
     if p.n_global > 0:
         prims.append(i < p.n_global or j < p.n_global)
     if p.block_local > 0:

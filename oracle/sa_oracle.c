@@ -20,6 +20,9 @@
  *    BigBird random blocks, blockwise (block-local) attention; and
  *    "Multi-Query and Grouped-Query Attention": H query heads share H_kv K/V
  *    heads (read as contiguous groups, h_kv = h / (H / H_kv)).
+ *    The same table's dilated/strided row ("every k-th token", O(N*w)) is read
+ *    as the window with its taps k apart: (i - j) mod k == 0 and the window
+ *    test applied to the tap number m = (i - j) / k.
  *  - "SAS: Sparse Attention Synthesizer" (kindchill), Step 5 component 2:
  *    patterns are combined from primitives by logical OR.
  *  - "Block Sparse Flash Attention" (montaan AI Radio), paper summary and
@@ -53,7 +56,10 @@ typedef struct {
     int32_t random_block;  /* granularity of random blocks (rows and keys)         */
     int32_t n_random;      /* random key blocks per (head, query block)            */
     const int32_t *random_table; /* [H][ceil(N/random_block)][n_random] or NULL   */
+    int32_t dilation;      /* window taps this far apart; 0 or 1: contiguous       */
 } ora_pattern_t;
+
+static int dilation_of(const ora_pattern_t *p) { return p->dilation > 1 ? p->dilation : 1; }
 
 /* Inputs are either raw bf16 bit patterns (kind 0), converted exactly to
  * double, or doubles (kind 1). */
@@ -81,10 +87,15 @@ int ora_visible(const ora_pattern_t *p, int N, int h, int i, int j)
     int any_primitive = 0, in = 0;
     if (p->window > 0) {
         any_primitive = 1;
-        if (p->causal) {
-            if (j >= i - p->window + 1 && j <= i) in = 1;
-        } else {
-            if (abs(i - j) <= p->window / 2) in = 1;
+        int k = dilation_of(p);
+        int dist = i - j;
+        if (dist % k == 0) {              /* j is one of the window's taps */
+            int m = dist / k;             /* tap number, 0 = the query itself */
+            if (p->causal) {
+                if (m >= 0 && m <= p->window - 1) in = 1;
+            } else {
+                if (abs(m) <= p->window / 2) in = 1;
+            }
         }
     }
     if (p->n_global > 0) {
@@ -121,7 +132,9 @@ int ora_build_G(const ora_pattern_t *p, int N, int h, int i, int32_t *out)
     int cap = 4 + (random_on(p) ? p->n_random : 0);
     range_t *r = (range_t *)malloc(sizeof(range_t) * cap);
     int nr = 0, any_primitive = 0;
-    if (p->window > 0) {
+    int dilated = p->window > 0 && dilation_of(p) > 1;   /* taps merged in below */
+    if (dilated) any_primitive = 1;
+    if (p->window > 0 && !dilated) {
         any_primitive = 1;
         if (p->causal) { r[nr].lo = (int64_t)i - p->window + 1; r[nr].hi = (int64_t)i + 1; }
         else           { r[nr].lo = (int64_t)i - p->window / 2; r[nr].hi = (int64_t)i + p->window / 2 + 1; }
@@ -165,6 +178,31 @@ int ora_build_G(const ora_pattern_t *p, int N, int h, int i, int32_t *out)
         if (hi > next) next = hi;
     }
     free(r);
+    if (dilated) {
+        /* the window's taps i + m*k, listed in ascending order, merged with the
+           (sorted, distinct) members emitted above */
+        int64_t k = dilation_of(p);
+        int64_t m_lo = p->causal ? -(int64_t)(p->window - 1) : -(int64_t)(p->window / 2);
+        int64_t m_hi = p->causal ? 0 : (int64_t)(p->window / 2);
+        int32_t *taps = (int32_t *)malloc(sizeof(int32_t) * (size_t)(m_hi - m_lo + 1));
+        int nt = 0;
+        for (int64_t m = m_lo; m <= m_hi; ++m) {
+            int64_t j = (int64_t)i + m * k;
+            if (j >= 0 && j < cap_hi) taps[nt++] = (int32_t)j;
+        }
+        int32_t *merged = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + nt + 1));
+        int a = 0, b = 0, c = 0;
+        while (a < n || b < nt) {
+            int32_t v;
+            if (b >= nt || (a < n && out[a] <= taps[b])) v = out[a++];
+            else v = taps[b++];
+            if (c == 0 || merged[c - 1] != v) merged[c++] = v;
+        }
+        memcpy(out, merged, sizeof(int32_t) * (size_t)c);
+        n = c;
+        free(merged);
+        free(taps);
+    }
     return n;
 }
 

@@ -1,0 +1,119 @@
+"""Dilated/strided sliding window (taps k apart) on the GPU.
+
+The kernels run a dilated window as k contiguous-window attentions, one per
+residue class i mod k, read through a strided TMA view.  Checked here: the
+result against the fp64 oracle's dilated predicate element by element (several
+tiles per class and ragged tails), bit equality with the contiguous-window
+kernel run on each class's rows copied out, the no-alloc entry point, and the
+combinations the kernels refuse.
+"""
+import numpy as np
+import pytest
+import torch
+
+from _parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _rand(shape, seed, device):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return torch.randn(shape, generator=g).to(torch.bfloat16).to(device)
+
+
+# (B, H, H_kv, N, d, causal, window taps, dilation); N / dilation positions per
+# class, several 128-row tiles with a ragged last one
+CASES = [
+    (1, 2, 1, 3 * 300, 64, 1, 100, 3),
+    (1, 4, 2, 2 * 1000, 128, 1, 256, 2),
+    (2, 2, 2, 8 * 200, 64, 0, 64, 8),
+    (1, 2, 2, 64 * 130, 128, 1, 40, 64),
+    (1, 2, 1, 5 * 777, 128, 0, 301, 5),
+    (1, 2, 2, 7 * 129, 128, 1, 1, 7),      # one tap: each row sees only itself
+    (1, 2, 2, 4 * 5, 64, 1, 3, 4),         # fewer positions per class than one block
+]
+
+
+def _inputs(B, H, Hkv, N, d, seed, cuda):
+    """Q, K ~ N(0,1); V ~ N(0,1)/4.  The first rows of every residue class see
+    only a few taps, so their softmax is close to one-hot and their output is
+    close to one V row.  With N(0,1) values such outputs pass |out| = 2, where
+    the bf16 output's own half-ulp (0.0078; 0.0156 above 4) plus the bf16
+    rounding of P exceed the 1e-2 budget whatever the kernel does (measured:
+    0.0100x at W = 40, k = 64).  At a quarter of the scale every output stays
+    below 2 and the budget holds; a wrong tap still moves rows by O(0.1)."""
+    return (_rand((B, H, N, d), seed, cuda), _rand((B, Hkv, N, d), seed + 1, cuda),
+            (_rand((B, Hkv, N, d), seed + 2, cuda).float() * 0.25).to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_dilated_window_matches_oracle(product, oracle_mod, cuda, case):
+    B, H, Hkv, N, d, causal, W, k = CASES[case]
+    Q, K, V = _inputs(B, H, Hkv, N, d, 300 + 11 * case, cuda)
+    pat = product.Pattern(causal=causal, window=W, dilation=k)
+    plan = product.Plan(pat, B, H, Hkv, N, d)
+    n = N // k
+    assert plan.info["T_q"] == -(-n // 128)
+    assert plan.info["n_units"] == B * k * H * (-(-n // 128))
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=cuda)
+    O = plan.prefill(Q, K, V, lse=lse)
+    product.check_device_error()
+    Or, lr = oracle_mod.prefill(oracle_mod.Pattern(causal=causal, window=W, dilation=k),
+                                Q.cpu(), K.cpu(), V.cpu())
+    assert_close(O, Or)
+    assert_close(lse, lr, what="lse")
+    # pair count of the plan = sum over rows of |G_i| of the dilated pattern
+    pairs = sum(len(oracle_mod.build_G(oracle_mod.Pattern(causal=causal, window=W, dilation=k),
+                                       N, 0, i)) for i in range(N))
+    assert plan.info["pairs"] == B * H * pairs
+
+
+@pytest.mark.parametrize("case", [0, 2, 3])
+def test_dilated_window_is_contiguous_window_per_class(product, cuda, case):
+    """Bit equality: the dilated launch's rows of class r are the bytes that the
+    contiguous-window kernel produces on that class's rows copied out."""
+    B, H, Hkv, N, d, causal, W, k = CASES[case]
+    Q, K, V = _inputs(B, H, Hkv, N, d, 500 + case, cuda)
+    O = product.Plan(product.Pattern(causal=causal, window=W, dilation=k), B, H, Hkv, N,
+                     d).prefill(Q, K, V)
+    plain = product.Plan(product.Pattern(causal=causal, window=W), B, H, Hkv, N // k, d)
+    for r in range(k):
+        Or = plain.prefill(Q[:, :, r::k].contiguous(), K[:, :, r::k].contiguous(),
+                           V[:, :, r::k].contiguous())
+        torch.cuda.synchronize()
+        assert torch.equal(O[:, :, r::k], Or), r
+    product.check_device_error()
+
+
+def test_dilated_window_one_shot_and_no_alloc(product, cuda):
+    B, H, Hkv, N, d, causal, W, k = CASES[1]
+    Q, K, V = _inputs(B, H, Hkv, N, d, 777, cuda)
+    pat = product.Pattern(causal=causal, window=W, dilation=k)
+    O1 = product.Plan(pat, B, H, Hkv, N, d).prefill(Q, K, V)
+    O2 = product.sparse_attn_prefill(Q, K, V, pat)
+    O3 = product.sparse_attn_prefill_noalloc(Q, K, V, pat, torch.empty_like(Q))
+    # the plan cache tells dilations apart
+    O4 = product.sparse_attn_prefill(Q, K, V, product.Pattern(causal=causal, window=W))
+    torch.cuda.synchronize()
+    product.check_device_error()
+    assert torch.equal(O1, O2) and torch.equal(O1, O3)
+    assert not torch.equal(O1, O4)
+
+
+def test_dilated_window_refusals(product, cuda):
+    B, H, Hkv, N, d = 1, 4, 2, 600, 128
+    Q, K, V = _inputs(B, H, Hkv, N, d, 9, cuda)
+    with pytest.raises(product.SparseAttnError):      # 7 does not divide N
+        product.Plan(product.Pattern(causal=1, window=8, dilation=7), B, H, Hkv, N, d)
+    with pytest.raises(product.SparseAttnError):      # combined with global tokens
+        product.Plan(product.Pattern(causal=1, window=8, dilation=3, n_global=2), B, H, Hkv, N, d)
+    with pytest.raises(product.SparseAttnError):      # paired-head kernel
+        product.Plan(product.Pattern(causal=1, window=8, dilation=3), B, H, Hkv, N, d,
+                     kernel=product.KERNEL_PAIRED_HEADS)
+    plan = product.Plan(product.Pattern(causal=1, window=8, dilation=3), B, H, Hkv, N, d)
+    thr = torch.zeros(H, dtype=torch.float32, device=cuda)
+    with pytest.raises(product.SparseAttnError):      # block-skip rule
+        plan.prefill(Q, K, V, thresholds=thr)
+    with pytest.raises(product.SparseAttnError):      # block statistics
+        plan.block_stats(Q, K)
+    product.check_device_error()

@@ -117,6 +117,13 @@ def _patterns(oracle_mod, N, H):
         P(causal=0, n_random=2, random_block=64, random_table=tab),
         P(causal=1, n_global=1, n_random=2, random_block=64, random_table=tab),
         P(causal=0, window=10, n_global=5, n_random=2, random_block=64, random_table=tab),
+        # dilated/strided windows (taps k apart), alone and in unions
+        P(causal=1, window=4, dilation=3),
+        P(causal=0, window=6, dilation=5),
+        P(causal=0, window=7, dilation=2),
+        P(causal=1, window=3, dilation=70),
+        P(causal=0, window=5, dilation=4, n_global=2),
+        P(causal=1, window=6, dilation=3, block_local=16),
     ]
 
 
@@ -140,6 +147,54 @@ def test_window_closed_form(oracle_mod):
     p = oracle_mod.Pattern(causal=1, window=W)
     for i in range(N):
         assert len(oracle_mod.build_G(p, N, 0, i)) == min(i + 1, W)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 7, 64])
+def test_dilated_window_closed_form(oracle_mod, k):
+    """Dilated window (W taps k apart): causal |G_i| = min(floor(i/k) + 1, W);
+    non-causal |G_i| = min(floor(i/k), W/2) + 1 + min(floor((N-1-i)/k), W/2);
+    every member j has (i - j) mod k == 0."""
+    N = 400
+    for W in (1, 5, 16):
+        pc = oracle_mod.Pattern(causal=1, window=W, dilation=k)
+        pn = oracle_mod.Pattern(causal=0, window=W, dilation=k)
+        for i in range(0, N, 7):
+            G = oracle_mod.build_G(pc, N, 0, i)
+            assert len(G) == min(i // k + 1, W)
+            assert np.all((i - G) % k == 0) and G.max() == i
+            Gn = oracle_mod.build_G(pn, N, 0, i)
+            assert len(Gn) == min(i // k, W // 2) + 1 + min((N - 1 - i) // k, W // 2)
+            assert np.all((i - Gn) % k == 0)
+
+
+def test_dilation_zero_and_one_are_the_contiguous_window(oracle_mod):
+    N = 200
+    for causal, W in ((1, 17), (0, 12)):
+        base = oracle_mod.Pattern(causal=causal, window=W)
+        for dil in (0, 1):
+            p = oracle_mod.Pattern(causal=causal, window=W, dilation=dil)
+            for i in range(N):
+                assert np.array_equal(oracle_mod.build_G(p, N, 0, i),
+                                      oracle_mod.build_G(base, N, 0, i))
+
+
+@pytest.mark.parametrize("causal", [1, 0])
+def test_dilated_window_is_window_on_residue_classes(oracle_mod, causal):
+    """A dilated window joins only positions of one residue class i mod k, and
+    inside a class (numbered m = i // k) it is the contiguous window: the
+    dilated attention's rows of class r equal the contiguous-window attention
+    over the subsequence r, r + k, r + 2k, ..."""
+    B, H, Hkv, N, d, k, W = 1, 2, 1, 3 * 41, 8, 3, 6
+    Q, K, V = _rand((B, H, N, d), 61), _rand((B, Hkv, N, d), 62), _rand((B, Hkv, N, d), 63)
+    O, lse = oracle_mod.prefill(oracle_mod.Pattern(causal=causal, window=W, dilation=k), Q, K, V)
+    for r in range(k):
+        sl = slice(r, None, k)
+        Or, lr = oracle_mod.prefill(oracle_mod.Pattern(causal=causal, window=W),
+                                    np.ascontiguousarray(Q[:, :, sl]),
+                                    np.ascontiguousarray(K[:, :, sl]),
+                                    np.ascontiguousarray(V[:, :, sl]), scale=1 / np.sqrt(d))
+        assert np.max(np.abs(O[:, :, sl] - Or)) < 1e-13
+        assert np.max(np.abs(lse[:, :, sl] - lr)) < 1e-12
 
 
 def test_tiny_static_pair_count(oracle_mod):

@@ -78,3 +78,36 @@ def test_workload_block_counts(product):
         product.Pattern(**w.pattern_fields()), w.H, w.N)
     assert int(row_ptr[-1]) == sum(2 * t + 2 for t in range(T)) == 65792
     assert int((~full).sum()) == 2 * T     # the two diagonal blocks of each tile
+
+
+@pytest.mark.parametrize("causal,W,k,N", [(1, 100, 3, 3 * 300), (0, 64, 8, 8 * 200),
+                                          (1, 40, 64, 64 * 130), (0, 301, 5, 5 * 257)])
+def test_dilated_lists_cover_every_residue_class(product, oracle_mod, causal, W, k, N):
+    """A dilated window compiles to the lists of one residue class: for every
+    class r, the oracle's G of row m*k + r, renumbered j -> (j - r) / k, gives
+    exactly the listed blocks and pair counts of tile m // 128."""
+    pat = product.Pattern(causal=causal, window=W, dilation=k)
+    row_ptr, kb, full, cnt, H_pat, T = product.compile_pattern(pat, 1, N)
+    n = N // k
+    assert H_pat == 1 and T == -(-n // 128)
+    op = oracle_mod.Pattern(causal=causal, window=W, dilation=k)
+    for r in sorted({0, k - 1, k // 2}):
+        for t in range(T):
+            exp = np.zeros(-(-n // 64), np.int64)
+            for m in range(t * 128, min(n, t * 128 + 128)):
+                G = oracle_mod.build_G(op, N, 0, m * k + r)
+                assert np.all((G - r) % k == 0)
+                np.add.at(exp, ((G - r) // k) // 64, 1)
+            lo, hi = row_ptr[t], row_ptr[t + 1]
+            assert np.array_equal(kb[lo:hi], np.nonzero(exp)[0]), (r, t)
+            assert np.array_equal(cnt[lo:hi], exp[kb[lo:hi]]), (r, t)
+
+
+@pytest.mark.parametrize("bad", [dict(causal=1, window=8, dilation=3, n_global=2),
+                                 dict(causal=0, window=8, dilation=2, block_local=64),
+                                 dict(causal=1, window=0, dilation=2),
+                                 dict(causal=1, window=8, dilation=7),   # 7 does not divide N
+                                 dict(causal=1, window=8, dilation=-1)])
+def test_dilated_window_rejections(product, bad):
+    with pytest.raises(product.SparseAttnError):
+        product.compile_pattern(product.Pattern(**bad), 1, 600)

@@ -147,8 +147,9 @@ def _sample_rows(B, H, N, n_random, seed):
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name,kernel", [("mistral_swa", 0), ("mistral_swa", 2),
-                                         ("longformer_bigbird", 0)],
-                         ids=["mistral_swa", "mistral_swa-paired", "longformer_bigbird"])
+                                         ("longformer_bigbird", 0), ("dilated_swa", 0)],
+                         ids=["mistral_swa", "mistral_swa-paired", "longformer_bigbird",
+                              "dilated_swa"])
 def test_prefill_full_size_sampled(product, oracle_mod, cuda, name, kernel):
     w = WORKLOADS[name]
     Q, K, V, tab = prefill_inputs(w, device=cuda)
