@@ -80,6 +80,8 @@ def _load():
         lib.ora_dense.argtypes = [i32, i32, i32, i32, i32, i32, dbl, i32, vp, vp, vp, vp]
         lib.ora_gather.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, dbl, vp, vp, vp,
                                    vp, vp, vp, vp, i32]
+        lib.ora_topk_select.argtypes = [i32, i32, i32, i32, i32, i32, dbl, vp, vp, vp, i32,
+                                        vp, vp, vp, vp, i32]
         _lib = lib
     return _lib
 
@@ -294,6 +296,33 @@ def gather(Q, K, V, idx, idx_len=None, scale=None, nthreads=0):
                        q.ctypes.data, k.ctypes.data, v.ctypes.data, ix.ctypes.data, _p(il),
                        O.ctypes.data, lse.ctypes.data, nthreads)
     return O, lse
+
+
+def topk_select(Q, K, top_k, lengths=None, scale=None, nthreads=0):
+    """Dynamic top-K sets of decode queries ("SAS", component 1, primitive C).
+
+    Q: [S][H][d]; K: [S][H_kv][L][d]; lengths: int [S] keys per sequence (or
+    None = L).  G of query (s, h) = the min(top_k, len_s) keys j < len_s with the
+    largest scale * q . k_j, ties to the smaller j.  Returns (idx int32
+    [S][H][top_k] ascending within the first idx_len entries, idx_len int32
+    [S][H], kth [S][H] smallest selected score, nxt [S][H] largest unselected
+    score; NaN where there is none).  Feed (idx, idx_len) to gather() for the
+    output.
+    """
+    kq, q = _as_input(Q)
+    kk, k = _as_input(K)
+    assert kq == kk
+    S, H, d = q.shape
+    Hkv, L = k.shape[1], k.shape[2]
+    ln = None if lengths is None else np.ascontiguousarray(lengths, dtype=np.int32)
+    idx = np.zeros((S, H, max(int(top_k), 1)), np.int32)
+    idx_len = np.zeros((S, H), np.int32)
+    kth = np.zeros((S, H), np.float64)
+    nxt = np.zeros((S, H), np.float64)
+    _load().ora_topk_select(kq, S, H, Hkv, L, d, default_scale(d) if scale is None else scale,
+                            q.ctypes.data, k.ctypes.data, _p(ln), int(top_k), idx.ctypes.data,
+                            idx_len.ctypes.data, kth.ctypes.data, nxt.ctypes.data, nthreads)
+    return idx[:, :, :top_k], idx_len, kth, nxt
 
 
 def block_stats(p: Pattern, Q, K, scale=None, tiles=None, nthreads=0):

@@ -23,6 +23,12 @@
  *    The same table's dilated/strided row ("every k-th token", O(N*w)) is read
  *    as the window with its taps k apart: (i - j) mod k == 0 and the window
  *    test applied to the tap number m = (i - j) / k.
+ *  - "SAS: Sparse Attention Synthesizer" (kindchill), Step 5 component 1,
+ *    primitive C ("attend to top-K dynamic tokens"), and the dynamic patterns
+ *    of "Sparse Attention Weights Assumption" (tokens with the highest
+ *    relevance scores): for one decode query, G = the top_k keys by relevance
+ *    score s_j = scale * q . k_j, ties to the smaller index (ora_topk_select);
+ *    the output is then the sparse output formula over that G.
  *  - "SAS: Sparse Attention Synthesizer" (kindchill), Step 5 component 2:
  *    patterns are combined from primitives by logical OR.
  *  - "Block Sparse Flash Attention" (montaan AI Radio), paper summary and
@@ -464,5 +470,66 @@ void ora_gather(int kind, int S, int H, int Hkv, int H_idx, int L, int d, int n_
         int nG = idx_len ? idx_len[(int64_t)s * H_idx + hi] : n_idx;
         row_attention(kind, Q, u * d, K, V, ((int64_t)s * Hkv + hkv) * L * d, d, scale,
                       G, nG, NULL, 0, O + u * d, lse + u);
+    }
+}
+
+/* ---- dynamic top-K selection for decode queries ----
+ * For query (s, h) over the keys j < len_s of its K/V head (len_s = lengths[s],
+ * or L): relevance s_j = scale * q . k_j in double; G = the k = min(top_k, len_s)
+ * keys with the largest s_j, equal scores ordered by the smaller j; written to
+ * idx_out[s][h][0..k) in ascending j, k to len_out[s][h].  kth_out[s][h] = the
+ * smallest selected score and next_out[s][h] = the largest unselected score
+ * (NAN when there is none), so a caller can tell how close the cut was. */
+typedef struct { double s; int32_t j; } ora_scored_t;
+
+static int cmp_scored_desc(const void *a, const void *b)
+{
+    const ora_scored_t *x = (const ora_scored_t *)a, *y = (const ora_scored_t *)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+static int cmp_i32(const void *a, const void *b)
+{
+    int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+void ora_topk_select(int kind, int S, int H, int Hkv, int L, int d, double scale,
+                     const void *Q, const void *K, const int32_t *lengths, int top_k,
+                     int32_t *idx_out, int32_t *len_out, double *kth_out, double *next_out,
+                     int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t u = 0; u < (int64_t)S * H; ++u) {
+        int s = (int)(u / H), h = (int)(u % H);
+        int hkv = h / (H / Hkv);
+        int len = lengths ? lengths[s] : L;
+        if (len < 0) len = 0;
+        if (len > L) len = L;
+        int k = top_k < len ? top_k : len;
+        int64_t kv_off = ((int64_t)s * Hkv + hkv) * L * d;
+        ora_scored_t *sc = (ora_scored_t *)malloc(sizeof(ora_scored_t) * (size_t)(len > 0 ? len : 1));
+        for (int j = 0; j < len; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += ld(Q, u * d + c, kind) * ld(K, kv_off + (int64_t)j * d + c, kind);
+            sc[j].s = scale * acc;
+            sc[j].j = j;
+        }
+        qsort(sc, (size_t)len, sizeof(ora_scored_t), cmp_scored_desc);
+        int32_t *out = idx_out + u * top_k;
+        for (int t = 0; t < k; ++t) out[t] = sc[t].j;
+        qsort(out, (size_t)k, sizeof(int32_t), cmp_i32);
+        len_out[u] = k;
+        kth_out[u] = k > 0 ? sc[k - 1].s : NAN;
+        next_out[u] = k < len ? sc[k].s : NAN;
+        free(sc);
     }
 }

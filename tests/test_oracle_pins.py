@@ -362,3 +362,89 @@ def test_bf16_inputs_convert_exactly(oracle_mod):
     O1, _ = oracle_mod.prefill(p, Qb, Kb, Vb)
     O2, _ = oracle_mod.prefill(p, Qb.double().numpy(), Kb.double().numpy(), Vb.double().numpy())
     assert np.array_equal(O1, O2)
+
+
+# ---------------------------------------------------------------- dynamic top-K
+def _decode_inputs(S, H, Hkv, L, d, seed):
+    return (_rand((S, H, d), seed), _rand((S, Hkv, L, d), seed + 1), _rand((S, Hkv, L, d), seed + 2))
+
+
+def test_topk_covering_every_key_is_dense_decode(oracle_mod):
+    """top_k >= len: G is every key j < len, so the output is the dense softmax
+    row (torch float64) of the query over those keys."""
+    import torch
+    S, H, Hkv, L, d = 2, 4, 2, 60, 16
+    Q, K, V = _decode_inputs(S, H, Hkv, L, d, 81)
+    lengths = np.array([60, 23])
+    idx, n, kth, nxt = oracle_mod.topk_select(Q, K, 64, lengths=lengths)
+    assert n.tolist() == [[60] * H, [23] * H] and np.all(np.isnan(nxt))
+    O, lse = oracle_mod.gather(Q, K, V, idx, n)
+    for s in range(S):
+        for h in range(H):
+            ln = lengths[s]
+            q = torch.from_numpy(Q[s, h])
+            k = torch.from_numpy(K[s, h // 2, :ln])
+            v = torch.from_numpy(V[s, h // 2, :ln])
+            w = torch.softmax(k @ q / np.sqrt(d), dim=0)
+            assert np.max(np.abs((w @ v).numpy() - O[s, h])) < 1e-12
+            assert abs(torch.logsumexp(k @ q / np.sqrt(d), 0).item() - lse[s, h]) < 1e-12
+
+
+def test_topk_recovers_planted_keys(oracle_mod):
+    """Keys built to score highest (a large multiple of the query direction
+    added to a chosen set P) are exactly the selected set."""
+    S, H, Hkv, L, d, k = 1, 2, 1, 500, 32, 37
+    Q, K, _ = _decode_inputs(S, H, Hkv, L, d, 82)
+    Q[0, 1] = Q[0, 0]                        # both heads share the query direction
+    P = np.sort(np.random.default_rng(5).choice(L, size=k, replace=False))
+    qd = Q[0, 0] / np.linalg.norm(Q[0, 0])
+    K[0, 0, P] += 40.0 * qd
+    idx, n, kth, nxt = oracle_mod.topk_select(Q, K, k)
+    for h in range(H):
+        assert n[0, h] == k and np.array_equal(idx[0, h, :k], P)
+        assert kth[0, h] > nxt[0, h]
+
+
+def test_topk_matches_sort_of_numpy_scores(oracle_mod):
+    """Against numpy: scores by einsum, order by (score desc, index asc) with
+    lexsort; random lengths, all GQA groupings."""
+    S, H, Hkv, L, d, k = 3, 8, 2, 300, 24, 41
+    Q, K, _ = _decode_inputs(S, H, Hkv, L, d, 83)
+    lengths = np.array([300, 41, 7])
+    idx, n, kth, nxt = oracle_mod.topk_select(Q, K, k, lengths=lengths, scale=0.3)
+    for s in range(S):
+        for h in range(H):
+            ln = lengths[s]
+            sc = 0.3 * np.einsum("jd,d->j", K[s, h // 4, :ln], Q[s, h])
+            order = np.lexsort((np.arange(ln), -sc))
+            want = np.sort(order[:min(k, ln)])
+            assert n[s, h] == len(want) and np.array_equal(idx[s, h, :n[s, h]], want)
+
+
+def test_topk_ties_go_to_the_smaller_index(oracle_mod):
+    """Equal scores (identical key rows) are taken in index order."""
+    S, H, Hkv, L, d = 1, 1, 1, 50, 8
+    Q, K, _ = _decode_inputs(S, H, Hkv, L, d, 84)
+    K[0, 0, :] = K[0, 0, 0]
+    K[0, 0, 30] = K[0, 0, 0] + Q[0, 0]       # the one strictly higher score
+    idx, n, kth, nxt = oracle_mod.topk_select(Q, K, 5)
+    assert idx[0, 0].tolist() == [0, 1, 2, 3, 30]
+
+
+def test_topk_sets_are_nested_and_exclude_the_rest(oracle_mod):
+    """Sets for growing top_k are nested; V rows outside G do not move the output."""
+    S, H, Hkv, L, d = 1, 2, 1, 200, 16
+    Q, K, V = _decode_inputs(S, H, Hkv, L, d, 85)
+    prev = set()
+    for k in (1, 5, 17, 64, 200):
+        idx, n, _, _ = oracle_mod.topk_select(Q, K, k)
+        cur = set(idx[0, 0, :n[0, 0]].tolist())
+        assert prev <= cur and len(cur) == k
+        prev = cur
+    idx, n, _, _ = oracle_mod.topk_select(Q, K, 20)
+    O1, _ = oracle_mod.gather(Q, K, V, idx, n)
+    out = np.setdiff1d(np.arange(L), idx[0, 0, :20])
+    V2 = V.copy()
+    V2[0, 0, out] += 100.0
+    O2, _ = oracle_mod.gather(Q, K, V2, idx, n)
+    assert np.max(np.abs(O1[0, 0] - O2[0, 0])) < 1e-14
