@@ -287,6 +287,45 @@ def setup_window_decode(w, device, torch, sa, workloads):
                 tensors=(Q, K, V, pos, O), pos=pos)
 
 
+def setup_topk_decode(w, device, torch, sa, workloads):
+    Q, K, V = workloads.topk_decode_inputs(w, device=device)
+    O = torch.empty_like(Q)
+    idx = torch.zeros((w.S, w.H, w.top_k), dtype=torch.int32, device=device)
+    n_sel = torch.zeros((w.S, w.H), dtype=torch.int32, device=device)
+    ws = torch.empty(sa.decode_topk_workspace_bytes(w.S, w.H, w.L, w.top_k), dtype=torch.uint8,
+                     device=device)
+    # every K row is scored once per (sequence, K/V head); the selected V rows
+    # are read once per (sequence, query head)
+    k_bytes = w.S * w.H_kv * w.L * w.d * 2
+    v_bytes = w.S * w.H * w.top_k * w.d * 2
+    algo_bytes = k_bytes + v_bytes + Q.numel() * 2 + O.numel() * 2
+    flops = 2 * w.S * w.H * w.L * w.d + 2 * w.S * w.H * w.top_k * w.d
+
+    def step(stream=None):
+        sa.sparse_attn_decode_topk(Q, K, V, w.top_k, O=O, idx=idx, idx_len=n_sel, workspace=ws,
+                                   stream=stream)
+
+    host = [Q.cpu().pin_memory(), torch.empty(O.shape, dtype=O.dtype, pin_memory=True)]
+    Qd, Od = torch.empty_like(Q), torch.empty_like(O)
+
+    def e2e_step(stream):
+        Qd.copy_(host[0], non_blocking=True)
+        sa.sparse_attn_decode_topk(Qd, K, V, w.top_k, O=Od, idx=idx, idx_len=n_sel, workspace=ws,
+                                   stream=stream)
+        host[1].copy_(Od, non_blocking=True)
+
+    h2d = host[0].numel() * 2
+    d2h = host[1].numel() * 2
+    return dict(step=step, e2e_step=e2e_step, h2d=h2d, d2h=d2h, flops=flops, exact_flops=flops,
+                dense_flops=flops, algo_bytes=algo_bytes,
+                extra={"k_bytes_scored": k_bytes, "v_bytes_selected": v_bytes,
+                       "workspace_bytes": ws.numel()},
+                kernel="topk_score_kernel", kernel_files=["topk_sm100.cu"],
+                launches_per_step=3,
+                metric="top-K decode GB/s", unit="GB/s", bound="hbm",
+                tensors=(Q, K, V, None, O))
+
+
 # ------------------------------------------------------------- CPU baseline --
 def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
     """Times the fp64 oracle as it stands on the host cores over a bounded sample
@@ -325,6 +364,26 @@ def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
             n = min(32, n * 2)
         gbs = done_rows * (2 * w.d * 2) / t_total / 1e9
         return gbs, cores, f"{done_rows // m} (sequence, head) queries, {done_rows} cache rows"
+    if isinstance(w, workloads.TopkDecodeWorkload):
+        # top-K decode: sampled (sequence, head) queries, each scored against its
+        # K/V head's whole cache, then attending to its selected keys
+        Q, K, V, _ = device_tensors
+        group = w.H // w.H_kv
+        done, t_total, scanned, picked = 0, 0.0, 0, 0
+        while t_total < seconds:
+            s, h = int(g.integers(w.S)), int(g.integers(w.H))
+            Qh = Q[s, h][None, None].cpu()
+            Kh = K[s, h // group][None, None].cpu()
+            Vh = V[s, h // group][None, None].cpu()
+            t0 = time.perf_counter()
+            ix, n, _, _ = oracle.topk_select(Qh, Kh, w.top_k, nthreads=cores)
+            oracle.gather(Qh, Kh, Vh, ix, n, nthreads=cores)
+            t_total += time.perf_counter() - t0
+            done += 1
+            scanned += w.L
+            picked += int(n[0, 0])
+        gbs = (scanned * w.d * 2 + picked * w.d * 2) / t_total / 1e9
+        return gbs, cores, f"{done} (sequence, head) queries over {w.L} keys each"
     if isinstance(w, workloads.GatherWorkload):
         # gather: sampled (sequence, head) sets, only their referenced rows on the host
         if device_tensors is None:
@@ -420,6 +479,8 @@ def main():
 
     if isinstance(w, workloads.WindowDecodeWorkload):
         setup = setup_window_decode
+    elif isinstance(w, workloads.TopkDecodeWorkload):
+        setup = setup_topk_decode
     else:
         setup = setup_gather if isinstance(w, workloads.GatherWorkload) else setup_prefill
     S = setup(w, device, torch, sa, workloads)
@@ -492,7 +553,7 @@ def main():
         "e2e": {"value": round(e2e_value, 3), "unit": S["unit"],
                 "h2d_bytes_per_step": S["h2d"], "d2h_bytes_per_step": S["d2h"],
                 "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * S.get("launches_per_step", 1),
         "roofline": {"bound": S["bound"], "achieved": round(achieved, 3), "peak": peak,
                      "unit": roof_unit, "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_src} ({'bf16_tflops burst' if roof_unit == 'TFLOP/s' else 'hbm_gbs'})",
@@ -513,7 +574,8 @@ def main():
                             "algorithmic_bytes": S["algo_bytes"], **S["extra"]}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        if isinstance(w, (workloads.GatherWorkload, workloads.WindowDecodeWorkload)):
+        if isinstance(w, (workloads.GatherWorkload, workloads.WindowDecodeWorkload,
+                          workloads.TopkDecodeWorkload)):
             Q, K, V, idx, _ = S["tensors"]
             dt = (Q, K, V, idx)
         else:
@@ -530,6 +592,10 @@ def main():
 
 def config_of(w, world):
     from block_sparse_attention_29_b200 import workloads
+    if isinstance(w, workloads.TopkDecodeWorkload):
+        return {"workload": w.name, "sequences": w.S, "H": w.H, "H_kv": w.H_kv, "d": w.d,
+                "cache_len": w.L, "top_k": w.top_k, "selection": "dynamic (scores at run time)",
+                "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}
     if isinstance(w, workloads.WindowDecodeWorkload):
         return {"workload": w.name, "sequences": w.S, "H": w.H, "H_kv": w.H_kv, "d": w.d,
                 "pattern": {"causal": 1, "window": w.window, "n_global": w.n_global},
@@ -557,6 +623,12 @@ def run_reference(args, w, world):
         ws = dataclasses.replace(w, S=4)
         dt = workloads.window_decode_inputs(ws, device="cpu")
         w = ws
+    elif isinstance(w, workloads.TopkDecodeWorkload):
+        import dataclasses
+        ws = dataclasses.replace(w, S=2)
+        Q, K, V = workloads.topk_decode_inputs(ws, device="cpu")
+        dt = (Q, K, V, None)
+        w = ws
     elif isinstance(w, workloads.GatherWorkload):
         # a cache of the full size does not fit the host budget of this arm: the
         # sampled sets' rows are drawn with the same recipe at reduced length
@@ -579,9 +651,11 @@ def run_reference(args, w, world):
         vals.append(v)
     elapsed = time.perf_counter() - t0
     value = statistics.mean(vals)
-    unit = ("GB/s" if isinstance(w, (workloads.GatherWorkload, workloads.WindowDecodeWorkload))
+    unit = ("GB/s" if isinstance(w, (workloads.GatherWorkload, workloads.WindowDecodeWorkload,
+                                     workloads.TopkDecodeWorkload))
             else "TFLOP/s")
     metric = ("window decode GB/s" if isinstance(w, workloads.WindowDecodeWorkload) else
+              "top-K decode GB/s" if isinstance(w, workloads.TopkDecodeWorkload) else
               "gather GB/s" if unit == "GB/s" else "effective TFLOP/s (computed blocks)")
     out = {"impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

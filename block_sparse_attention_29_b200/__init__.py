@@ -28,7 +28,8 @@ from ._lib import (EXPORTS, LIB_PATH, SA_ERR_DEVICE_INDEX, SA_ERR_INVALID_ARG, S
 
 __all__ = ["Pattern", "Plan", "KERNEL_AUTO", "KERNEL_SINGLE_HEAD", "KERNEL_PAIRED_HEADS",
            "sparse_attn_prefill", "sparse_attn_prefill_noalloc",
-           "sparse_attn_gather", "sparse_attn_decode_window", "window_slot", "compile_pattern",
+           "sparse_attn_gather", "sparse_attn_decode_window", "window_slot",
+           "sparse_attn_decode_topk", "decode_topk_workspace_bytes", "compile_pattern",
            "check_device_error", "SparseAttnError", "EXPORTS", "LIB_PATH", "SA_OK",
            "SA_ERR_INVALID_ARG", "SA_ERR_UNSUPPORTED", "SA_ERR_TIMEOUT", "SA_ERR_DEVICE_INDEX"]
 
@@ -258,6 +259,50 @@ def sparse_attn_decode_window(Q, K, V, positions, pattern: Pattern, O=None, lse=
     check(lib().sparse_attn_decode_window(_ptr(Q), _ptr(K), _ptr(V), _ptr(positions), _ptr(O), S,
                                           H, Hkv, d, ctypes.byref(st), _ptr(lse), _stream(stream)))
     return O
+
+
+def decode_topk_workspace_bytes(S: int, H: int, L: int, top_k: int) -> int:
+    """Workspace bytes sparse_attn_decode_topk needs for these sizes."""
+    return int(lib().sparse_attn_decode_topk_workspace(int(S), int(H), int(L), int(top_k)))
+
+
+def sparse_attn_decode_topk(Q, K, V, top_k: int, lengths=None, O=None, lse=None, idx=None,
+                            idx_len=None, scale: float = 0.0, workspace=None, stream=None):
+    """Decode attention over each query's top_k keys by relevance score.
+
+    Q [S][H][d]; K/V [S][H_kv][L][d]; lengths int32 [S] (keys per sequence) or
+    None.  Returns (O [S][H][d], idx int32 [S][H][top_k], idx_len int32 [S][H]):
+    the selected keys of (s, h) are idx[s, h, :idx_len[s, h]], ascending.
+    workspace: a uint8 device tensor of decode_topk_workspace_bytes(...) bytes
+    (allocated here when None)."""
+    import torch
+    S, H, d = Q.shape
+    Hkv, L = K.shape[1], K.shape[2]
+    _check_tensor("Q", Q, (S, H, d), torch.bfloat16)
+    _check_tensor("K", K, (S, Hkv, L, d), torch.bfloat16)
+    _check_tensor("V", V, (S, Hkv, L, d), torch.bfloat16)
+    if lengths is not None:
+        _check_tensor("lengths", lengths, (S,), torch.int32)
+    if O is None:
+        O = torch.empty_like(Q)
+    _check_tensor("O", O, (S, H, d), torch.bfloat16)
+    if lse is not None:
+        _check_tensor("lse", lse, (S, H), torch.float32)
+    if idx is None:
+        idx = torch.zeros((S, H, top_k), dtype=torch.int32, device=Q.device)
+    _check_tensor("idx", idx, (S, H, top_k), torch.int32)
+    if idx_len is None:
+        idx_len = torch.zeros((S, H), dtype=torch.int32, device=Q.device)
+    _check_tensor("idx_len", idx_len, (S, H), torch.int32)
+    need = decode_topk_workspace_bytes(S, H, L, top_k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    check(lib().sparse_attn_decode_topk(_ptr(Q), _ptr(K), _ptr(V), _ptr(lengths), _ptr(O), S, H,
+                                        Hkv, L, d, int(top_k), float(scale), _ptr(idx),
+                                        _ptr(idx_len), _ptr(lse), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)))
+    return O, idx, idx_len
 
 
 def window_slot(j: int, window: int, n_global: int) -> int:

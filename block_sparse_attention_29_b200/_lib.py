@@ -28,6 +28,7 @@ EXPORTS = (
     "sparse_attn_calibrate", "sparse_attn_gather", "sparse_attn_decode_window",
     "sparse_attn_window_slot", "sparse_attn_compile_pattern",
     "sparse_attn_check_device_error", "sparse_attn_last_error", "sparse_attn_prefill_noalloc",
+    "sparse_attn_decode_topk", "sparse_attn_decode_topk_workspace",
 )
 
 
@@ -84,7 +85,9 @@ def lib():
         L.sparse_attn_calibrate.argtypes = [vp, vp, f64, vp, vp]
         L.sparse_attn_decode_window.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, P, vp, vp]
         L.sparse_attn_window_slot.argtypes = [i64, i32, i32]
-        L.sparse_attn_window_slot.restype = i64
+        L.sparse_attn_decode_topk.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                              f32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.sparse_attn_decode_topk_workspace.argtypes = [i32, i32, i32, i32]
         L.sparse_attn_gather.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                          i32, f32, vp, vp]
         L.sparse_attn_compile_pattern.argtypes = [P, i32, i32, i32, i32,
@@ -97,6 +100,8 @@ def lib():
         for name in EXPORTS:
             if name not in ("sparse_attn_plan_destroy", "sparse_attn_last_error"):
                 getattr(L, name).restype = ctypes.c_int
+        L.sparse_attn_window_slot.restype = i64
+        L.sparse_attn_decode_topk_workspace.restype = ctypes.c_size_t
         _lib = L
     return _lib
 

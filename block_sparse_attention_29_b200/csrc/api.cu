@@ -559,6 +559,84 @@ int sparse_attn_decode_window(const void* Q, const void* K, const void* V,
   return launch_gather(p, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+namespace {
+// Workspace of the top-k decode: scores [S*H][Lp] fp32, first-level
+// histograms [S*H][kTopkBins1], selected keys [S*H][top_k] and counts [S*H];
+// each region starts on a 256-byte boundary.
+struct TopkLayout {
+  size_t scores = 0, hist = 0, idx = 0, idx_len = 0, total = 0;
+};
+size_t round_up256(size_t n) { return (n + 255) & ~size_t(255); }
+bool topk_layout(int S, int H, int L, int top_k, TopkLayout* t) {
+  if (S < 0 || H <= 0 || L <= 0 || top_k <= 0) return false;
+  const size_t sh = size_t(S) * size_t(H);
+  const size_t Lp = (size_t(L) + 3) & ~size_t(3);
+  t->scores = 0;
+  t->hist = round_up256(sh * Lp * 4);
+  t->idx = t->hist + round_up256(sh * kTopkBins1 * 4);
+  t->idx_len = t->idx + round_up256(sh * size_t(top_k) * 4);
+  t->total = t->idx_len + round_up256(sh * 4);
+  return true;
+}
+}  // namespace
+
+extern "C" {
+
+size_t sparse_attn_decode_topk_workspace(int S, int H, int L, int top_k) {
+  TopkLayout t;
+  return topk_layout(S, H, L, top_k, &t) ? t.total : 0;
+}
+
+int sparse_attn_decode_topk(const void* Q, const void* K, const void* V, const int32_t* lengths,
+                            void* O, int S, int H, int H_kv, int L, int d, int top_k, float scale,
+                            int32_t* idx_out, int32_t* idx_len_out, float* lse_out,
+                            void* workspace, size_t workspace_bytes, sa_stream_t stream) {
+  if (!Q || !K || !V || !O || !workspace)
+    return set_error(SA_ERR_INVALID_ARG, "Q, K, V, O and workspace must be non-NULL");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(workspace))
+    return set_error(SA_ERR_INVALID_ARG, "Q, K, V, O and workspace must be 16-byte aligned");
+  if (S < 0 || H <= 0 || H_kv <= 0 || L <= 0)
+    return set_error(SA_ERR_INVALID_ARG, "bad shape (S=%d H=%d H_kv=%d L=%d)", S, H, H_kv, L);
+  if (H % H_kv != 0) return set_error(SA_ERR_INVALID_ARG, "H = %d is not a multiple of H_kv = %d", H, H_kv);
+  if (top_k < 1) return set_error(SA_ERR_INVALID_ARG, "top_k = %d (must be >= 1)", top_k);
+  if (d != 64 && d != 128) return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
+  if (int64_t(S) * H > INT32_MAX || L > (1 << 29))
+    return set_error(SA_ERR_UNSUPPORTED, "S*H or L too large for the launch grids");
+  TopkLayout t;
+  topk_layout(S, H, L, top_k, &t);
+  if (workspace_bytes < t.total)
+    return set_error(SA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes,
+                     t.total);
+  if (S == 0) return SA_OK;
+  unsigned char* w = static_cast<unsigned char*>(workspace);
+  TopkParams p;
+  std::memset(&p, 0, sizeof p);
+  p.Q = static_cast<const uint16_t*>(Q);
+  p.K = static_cast<const uint16_t*>(K);
+  p.V = static_cast<const uint16_t*>(V);
+  p.lengths = lengths;
+  p.O = static_cast<uint16_t*>(O);
+  p.lse = lse_out;
+  p.scores = reinterpret_cast<float*>(w + t.scores);
+  p.hist = reinterpret_cast<uint32_t*>(w + t.hist);
+  p.idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + t.idx);
+  p.idx_len = idx_len_out ? idx_len_out : reinterpret_cast<int32_t*>(w + t.idx_len);
+  p.S = S;
+  p.H = H;
+  p.Hkv = H_kv;
+  p.L = L;
+  p.Lp = (L + 3) & ~3;
+  p.top_k = top_k;
+  p.chunk = kTopkChunk;
+  const float sc = scale != 0.f ? scale : 1.0f / sqrtf(float(d));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.err = device_error_word();
+  if (!p.err) return set_error(SA_ERR_CUDA, "device error word unavailable");
+  return launch_topk(p, d, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int64_t sparse_attn_window_slot(int64_t j, int window, int n_global) {
   if (j < 0 || window < 1 || n_global < 0) return -1;
   return j < n_global ? j : n_global + (j % window);

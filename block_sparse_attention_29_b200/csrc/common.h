@@ -102,6 +102,29 @@ struct GatherParams {
 
 int launch_gather(const GatherParams& p, int d, cudaStream_t stream);
 
+// ------------------------------------------------------------------ top-k --
+constexpr int kTopkBins1 = 2048;   // first-level histogram: the top 11 bits of a score's key
+constexpr int kTopkChunk = 8192;   // keys per CTA of the score pass
+
+struct TopkParams {
+  const uint16_t* Q;         // [S][H][d]
+  const uint16_t* K;         // [S][H_kv][L][d]
+  const uint16_t* V;
+  const int32_t* lengths;    // [S] keys per sequence, or null (all L)
+  uint16_t* O;               // [S][H][d]
+  float* lse;                // [S][H] or null
+  float* scores;             // workspace [S][H][Lp]: log2-scaled scores
+  uint32_t* hist;            // workspace [S][H][kTopkBins1]
+  int32_t* idx;              // [S][H][top_k] selected keys, ascending
+  int32_t* idx_len;          // [S][H] selected count
+  int S, H, Hkv, L, Lp, top_k, chunk;   // Lp: L rounded up to a multiple of 4
+  float scale_log2;
+  int* err;                  // device error word
+};
+
+// Score pass, radix select and attention over the selected keys.
+int launch_topk(const TopkParams& p, int d, cudaStream_t stream);
+
 // ------------------------------------------------------------ calibration --
 // Per-head rank selection over the statistics of full blocks (plan lists).
 int launch_calibrate(const float* stat, const int32_t* row_ptr, const int32_t* entries,

@@ -1,0 +1,478 @@
+// topk_sm100.cu -- decode attention over the top_k keys of each query: the
+// dynamic primitive "attend to the top-K dynamic tokens" ("SAS: Sparse
+// Attention Synthesizer", Step 5, component 1, primitive C; the dynamic
+// patterns of "Sparse Attention Weights Assumption": tokens with the highest
+// relevance scores).  For query (s, h) over keys j < len_s of its K/V head:
+// score s_j = scale * q . k_j, G = the top_k keys by score (equal scores to
+// the smaller j), out = softmax over G of s_j, weighted sum of v_j.
+//
+// Three launches, each bound by HBM:
+//   1. score: one CTA per (chunk of 8192 keys, sequence, group of query heads
+//      sharing a K/V head).  Every K row is read once for all the heads of
+//      its group (16-byte loads, d/8 lanes per row), each score is written to
+//      the workspace (log2-scaled, fp32) and counted in a per-head histogram
+//      of the top 11 bits of its order-preserving key, kept in shared memory
+//      and added to global memory once per CTA.
+//   2. select: one CTA per (sequence, head) -- an exact radix select: the
+//      histogram gives the 11-bit bin of the top_k-th largest key, two passes
+//      over the head's scores resolve the next 11 and the last 10 bits, and a
+//      last pass writes the selected indices in ascending order (block-wide
+//      prefix sums), taking equal keys in index order.
+//   3. attend: one CTA per (sequence, head) -- online softmax over the stored
+//      scores of the selected keys and the weighted sum of their V rows.
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "common.h"
+#include "ptx.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int kSelectThreads = 1024;
+constexpr int kAttendThreads = 256;
+constexpr int kAttendUnroll = 8;
+
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f[2 * k] = __uint_as_float(w[k] << 16);
+    f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+
+// Order-preserving key of a score: unsigned comparison of keys is the
+// comparison of the floats (-0 is taken as +0, so equal floats give equal keys).
+__device__ __forceinline__ uint32_t topk_key(float x) {
+  const uint32_t u = __float_as_uint(x == 0.f ? 0.f : x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Keys of sequence s: lengths[s] clamped to [0, L] (an out-of-range length is
+// recorded as SA_ERR_DEVICE_INDEX at `site`).
+__device__ __forceinline__ int seq_len(const TopkParams& p, int s, int site) {
+  if (!p.lengths) return p.L;
+  const int n = __ldg(p.lengths + s);
+  if (n < 0 || n > p.L) {
+    if (threadIdx.x == 0) record_device_error(p.err, SA_ERR_DEVICE_INDEX, site);
+    return n < 0 ? 0 : p.L;
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------- score --
+// CTA: 8 warps; a row of D bf16 is read by LPR = D/8 lanes (16 bytes each), so
+// a warp step covers 32/LPR rows and a warp takes U steps per iteration (U
+// rows' loads in flight per lane).  Each lane ends a step with partial dot
+// products for its 8 dimensions, U*G of them per iteration; they are summed
+// over the row's LPR lanes by a transposing reduction: at each of the
+// log2(LPR) exchange steps a lane keeps half of its values, sends the other
+// half to its partner and adds what it receives, so V values cost V-1
+// shuffles in all instead of V*log2(LPR), and lane l of a row ends holding
+// the totals l*(V/LPR) .. l*(V/LPR) + V/LPR - 1 (value index = u*G + g).
+template <int D, int G>
+struct ScoreCfg {
+  static constexpr int LPR = D / 8;
+  static constexpr int RPS = 32 / LPR;                  // rows per warp step
+  static constexpr int U = (32 / G) > 16 ? 16 : 32 / G;  // steps per iteration
+  static constexpr int V = U * G;                        // partial dots per lane
+  static constexpr int HV = V / LPR;                     // totals per lane
+  static constexpr int ROWS_WARP = RPS * U;
+  static constexpr int ROWS_IT = ROWS_WARP * (kScoreThreads / 32);
+  static_assert(V % LPR == 0 && V >= LPR, "reduction needs V a multiple of LPR");
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(kScoreThreads, 2) topk_score_kernel(const TopkParams p) {
+  using C = ScoreCfg<D, G>;
+  extern __shared__ uint32_t hist[];   // [G][kTopkBins1]
+  const int nqg = p.H / G;
+  const int s = blockIdx.x / nqg, qg = blockIdx.x % nqg;
+  const int h0 = qg * G;                      // first query head of the CTA
+  const int hkv = h0 / (p.H / p.Hkv);
+  const int len = seq_len(p, s, 3);
+  const int row_lo = blockIdx.y * p.chunk;
+  const int row_hi = min(len, row_lo + p.chunk);
+  if (row_lo >= row_hi) return;
+
+  for (int t = threadIdx.x; t < G * kTopkBins1; t += kScoreThreads) hist[t] = 0;
+  __syncthreads();
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int l = lane % C::LPR, slot = lane / C::LPR;
+  float q[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const uint4 qv =
+        *reinterpret_cast<const uint4*>(p.Q + ((int64_t)s * p.H + h0 + g) * D + l * 8);
+    bf16x8_to_f32(qv, q[g]);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) q[g][c] *= p.scale_log2;
+  }
+  const uint16_t* Kb = p.K + ((int64_t)s * p.Hkv + hkv) * p.L * D + l * 8;
+  float* Sb = p.scores + ((int64_t)s * p.H + h0) * p.Lp;
+
+  for (int base = row_lo + warp * C::ROWS_WARP; base < row_hi; base += C::ROWS_IT) {
+    uint4 kv[C::U];
+#pragma unroll
+    for (int u = 0; u < C::U; ++u) {
+      const int j = base + u * C::RPS + slot;
+      kv[u] = j < row_hi ? ld_stream(Kb + (int64_t)j * D) : make_uint4(0, 0, 0, 0);
+    }
+    float v[C::V];
+#pragma unroll
+    for (int u = 0; u < C::U; ++u) {
+      float kf[8];
+      bf16x8_to_f32(kv[u], kf);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float d = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) d = fmaf(q[g][c], kf[c], d);
+        v[u * G + g] = d;
+      }
+    }
+    // transposing reduction over the LPR lanes of each row
+#pragma unroll
+    for (int o = C::LPR / 2, half = C::V / 2; o > 0; o >>= 1, half >>= 1) {
+      const bool upper = (l & o) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float keep = upper ? v[half + i] : v[i];
+        const float send = upper ? v[i] : v[half + i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < C::HV; ++i) {
+      const int vi = l * C::HV + i;
+      const int u = vi / G, g = vi % G;
+      const int j = base + u * C::RPS + slot;
+      if (j < row_hi) {
+        Sb[(int64_t)g * p.Lp + j] = v[i];
+        atomicAdd(&hist[g * kTopkBins1 + (topk_key(v[i]) >> 21)], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  uint32_t* gh = p.hist + ((int64_t)s * p.H + h0) * kTopkBins1;
+  for (int t = threadIdx.x; t < G * kTopkBins1; t += kScoreThreads) {
+    const uint32_t c = hist[t];
+    if (c) atomicAdd(gh + t, c);
+  }
+}
+
+// --------------------------------------------------------------- select --
+// Exclusive prefix sum over the block (kSelectThreads threads); *total gets
+// the block's sum.  ws: shared [33].  Every thread must call it.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t* ws, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) ws[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t w = ws[lane];
+    uint32_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    ws[lane] = wi - w;
+    if (lane == 31) ws[32] = wi;
+  }
+  __syncthreads();
+  const uint32_t r = ws[warp] + inc - x;
+  *total = ws[32];
+  __syncthreads();
+  return r;
+}
+
+// The bin that holds the r-th largest key (r >= 1) of a histogram of NB bins,
+// bins taken from the top: above(b) < r <= above(b) + h[b].  Writes the bin and
+// the rank left inside it (r - above(b)) to res[0..1]; res[0] stays -1 when
+// the histogram holds fewer than r keys.
+template <int NB>
+__device__ __forceinline__ void find_bin(const uint32_t* h, uint32_t r, uint32_t* ws, int* res) {
+  constexpr int PER = NB / kSelectThreads;
+  if (threadIdx.x == 0) res[0] = -1;
+  uint32_t c[PER], sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    c[i] = h[NB - 1 - (threadIdx.x * PER + i)];
+    sum += c[i];
+  }
+  uint32_t total;
+  uint32_t above = block_excl_scan(sum, ws, &total);   // synchronises (res[0] visible)
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    if (above < r && r <= above + c[i]) {
+      res[0] = NB - 1 - (threadIdx.x * PER + i);
+      res[1] = int(r - above);
+    }
+    above += c[i];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(const TopkParams p) {
+  __shared__ uint32_t h[kTopkBins1];
+  __shared__ uint32_t ws[33];
+  __shared__ int res[2];
+  const int sh = blockIdx.x;
+  const int s = sh / p.H;
+  const int len = seq_len(p, s, 4);
+  const int k = min(p.top_k, len);
+  int32_t* out = p.idx + (int64_t)sh * p.top_k;
+  if (k == len) {   // every key is selected
+    for (int j = threadIdx.x; j < len; j += kSelectThreads) out[j] = j;
+    if (threadIdx.x == 0) p.idx_len[sh] = len;
+    return;
+  }
+  const float* sc = p.scores + (int64_t)sh * p.Lp;
+
+  // level 1: top 11 bits, from the score pass's histogram
+  for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads)
+    h[i] = p.hist[(int64_t)sh * kTopkBins1 + i];
+  __syncthreads();
+  find_bin<kTopkBins1>(h, uint32_t(k), ws, res);
+  const int b1 = res[0];
+  const uint32_t r1 = uint32_t(res[1]);
+  __syncthreads();
+  if (b1 < 0) {   // the histogram does not hold len keys: inconsistent workspace
+    if (threadIdx.x == 0) {
+      record_device_error(p.err, SA_ERR_DEVICE_INDEX, 5);
+      p.idx_len[sh] = 0;
+    }
+    return;
+  }
+  // level 2: bits 20..10 of the keys in bin b1
+  for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads) h[i] = 0;
+  __syncthreads();
+  for (int j0 = threadIdx.x * 4; j0 < len; j0 += kSelectThreads * 4) {
+    const float4 f = *reinterpret_cast<const float4*>(sc + j0);   // rows padded to Lp
+    const float x[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t key = topk_key(x[i]);
+      if (j0 + i < len && (key >> 21) == uint32_t(b1)) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+    }
+  }
+  __syncthreads();
+  find_bin<kTopkBins1>(h, r1, ws, res);
+  const int b2 = res[0];
+  const uint32_t r2 = uint32_t(res[1]);
+  __syncthreads();
+  // level 3: bits 9..0 of the keys with prefix (b1, b2)
+  const uint32_t pre = (uint32_t(b1) << 11) | uint32_t(b2 < 0 ? 0 : b2);
+  for (int i = threadIdx.x; i < 1024; i += kSelectThreads) h[i] = 0;
+  __syncthreads();
+  for (int j0 = threadIdx.x * 4; j0 < len; j0 += kSelectThreads * 4) {
+    const float4 f = *reinterpret_cast<const float4*>(sc + j0);
+    const float x[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t key = topk_key(x[i]);
+      if (j0 + i < len && (key >> 10) == pre) atomicAdd(&h[key & 1023u], 1u);
+    }
+  }
+  __syncthreads();
+  find_bin<1024>(h, r2, ws, res);
+  const int b3 = res[0];
+  const uint32_t take_eq = uint32_t(res[1]);   // keys equal to the threshold to take
+  __syncthreads();
+  if (b2 < 0 || b3 < 0) {
+    if (threadIdx.x == 0) {
+      record_device_error(p.err, SA_ERR_DEVICE_INDEX, 5);
+      p.idx_len[sh] = 0;
+    }
+    return;
+  }
+  const uint32_t thr = (pre << 10) | uint32_t(b3);
+
+  // output: keys above the threshold and the first take_eq equal ones, in
+  // ascending index order
+  uint32_t n_out = 0, n_eq = 0;
+  for (int c0 = 0; c0 < len; c0 += kSelectThreads * 4) {
+    const int j0 = c0 + threadIdx.x * 4;
+    bool gt[4], eq[4];
+    uint32_t ce = 0;
+    if (j0 < len) {
+      const float4 f = *reinterpret_cast<const float4*>(sc + j0);
+      const float x[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t key = topk_key(x[i]);
+        const bool in = j0 + i < len;
+        gt[i] = in && key > thr;
+        eq[i] = in && key == thr;
+        ce += eq[i];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) gt[i] = eq[i] = false;
+    }
+    uint32_t eq_total;
+    uint32_t eq_rank = n_eq + block_excl_scan(ce, ws, &eq_total);
+    bool sel[4];
+    uint32_t cs = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sel[i] = gt[i] || (eq[i] && eq_rank < take_eq);
+      eq_rank += eq[i];
+      cs += sel[i];
+    }
+    uint32_t sel_total;
+    uint32_t pos = n_out + block_excl_scan(cs, ws, &sel_total);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (sel[i] && pos < uint32_t(k)) out[pos++] = j0 + i;
+    n_out += sel_total;
+    n_eq += eq_total;
+  }
+  if (threadIdx.x == 0) {
+    if (n_out != uint32_t(k)) record_device_error(p.err, SA_ERR_DEVICE_INDEX, 6);
+    p.idx_len[sh] = int(min(n_out, uint32_t(k)));
+  }
+}
+
+// --------------------------------------------------------------- attend --
+// One CTA per (sequence, head): rows of the selected set split over row
+// groups of D/8 lanes; each group keeps an online softmax over the stored
+// scores (already log2-scaled) and accumulates its V rows; groups merge
+// through shared memory.
+template <int D>
+__global__ void __launch_bounds__(kAttendThreads) topk_attend_kernel(const TopkParams p) {
+  constexpr int LPR = D / 8;
+  constexpr int NG = kAttendThreads / LPR;
+  __shared__ float sm_m[NG], sm_l[NG];
+  __shared__ float sm_acc[NG][D];
+  const int sh = blockIdx.x;
+  const int s = sh / p.H, h = sh % p.H;
+  const int hkv = h / (p.H / p.Hkv);
+  const int grp = threadIdx.x / LPR, gl = threadIdx.x % LPR;
+  const int len = p.idx_len[sh];
+  const int32_t* idx = p.idx + (int64_t)sh * p.top_k;
+  const float* sc = p.scores + (int64_t)sh * p.Lp;
+  const uint16_t* Vb = p.V + ((int64_t)s * p.Hkv + hkv) * p.L * D + gl * 8;
+
+  float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  for (int base = grp; base < len; base += NG * kAttendUnroll) {
+    uint4 vv[kAttendUnroll];
+    float w[kAttendUnroll];
+#pragma unroll
+    for (int u = 0; u < kAttendUnroll; ++u) {
+      const int r = base + u * NG;
+      int j = r < len ? __ldg(idx + r) : -1;
+      if (j >= p.L) j = -1;   // cannot happen: the select pass writes indices < len
+      vv[u] = j >= 0 ? ld_stream(Vb + (int64_t)j * D) : make_uint4(0, 0, 0, 0);
+      w[u] = j >= 0 ? __ldg(sc + j) : -INFINITY;
+    }
+    float mx = w[0];
+#pragma unroll
+    for (int u = 1; u < kAttendUnroll; ++u) mx = fmaxf(mx, w[u]);
+    const float m_new = fmaxf(m, mx);
+    if (m_new == -INFINITY) continue;
+    const float alpha = ex2(m - m_new);
+    l *= alpha;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] *= alpha;
+    m = m_new;
+#pragma unroll
+    for (int u = 0; u < kAttendUnroll; ++u) {
+      const float pw = ex2(w[u] - m);
+      l += pw;
+      float vf[8];
+      bf16x8_to_f32(vv[u], vf);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = fmaf(pw, vf[c], acc[c]);
+    }
+  }
+  if (gl == 0) {
+    sm_m[grp] = m;
+    sm_l[grp] = l;
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) sm_acc[grp][gl * 8 + c] = acc[c];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float M = -INFINITY;
+    for (int g = 0; g < NG; ++g) M = fmaxf(M, sm_m[g]);
+    float L = 0.f, o = 0.f;
+    if (M != -INFINITY) {
+      for (int g = 0; g < NG; ++g) {
+        const float wg = ex2(sm_m[g] - M);
+        L = fmaf(sm_l[g], wg, L);
+        o = fmaf(sm_acc[g][threadIdx.x], wg, o);
+      }
+    }
+    const float out = L > 0.f ? o / L : 0.f;
+    p.O[(int64_t)sh * D + threadIdx.x] = __bfloat16_as_ushort(__float2bfloat16_rn(out));
+    if (threadIdx.x == 0 && p.lse)
+      p.lse[sh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+template <int D, int G>
+int launch_score(const TopkParams& p, cudaStream_t stream) {
+  const size_t smem = size_t(G) * kTopkBins1 * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(topk_score_kernel<D, G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute(topk score)");
+  }
+  const dim3 grid((unsigned)(p.S * (p.H / G)), (unsigned)((p.L + p.chunk - 1) / p.chunk));
+  topk_score_kernel<D, G><<<grid, kScoreThreads, smem, stream>>>(p);
+  return SA_OK;
+}
+
+}  // namespace
+
+int launch_topk(const TopkParams& p, int d, cudaStream_t stream) {
+  const int64_t n = (int64_t)p.S * p.H;
+  if (n == 0) return SA_OK;
+  if (d != 64 && d != 128) return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
+  const int group = p.H / p.Hkv;
+  // query heads scored together: a whole K/V group when it has 1, 2, 4 or 8
+  // heads, else one head per CTA (each CTA then reads its K/V head itself)
+  const int G = (group == 1 || group == 2 || group == 4 || group == 8) ? group : 1;
+  cudaError_t e = cudaMemsetAsync(p.hist, 0, size_t(n) * kTopkBins1 * sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return cuda_error(e, "cudaMemsetAsync(top-k histogram)");
+  int rc;
+#define SA_SCORE(DD)                                       \
+  switch (G) {                                             \
+    case 8: rc = launch_score<DD, 8>(p, stream); break;    \
+    case 4: rc = launch_score<DD, 4>(p, stream); break;    \
+    case 2: rc = launch_score<DD, 2>(p, stream); break;    \
+    default: rc = launch_score<DD, 1>(p, stream); break;   \
+  }
+  if (d == 128) { SA_SCORE(128) } else { SA_SCORE(64) }
+#undef SA_SCORE
+  if (rc) return rc;
+  topk_select_kernel<<<(unsigned)n, kSelectThreads, 0, stream>>>(p);
+  if (d == 128) topk_attend_kernel<128><<<(unsigned)n, kAttendThreads, 0, stream>>>(p);
+  else topk_attend_kernel<64><<<(unsigned)n, kAttendThreads, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_error(e, "top-k launch");
+  return SA_OK;
+}
+
+}  // namespace sa

@@ -23,6 +23,8 @@ Workloads (names used by tests and bench):
                       4 global tokens over a cache of 4100 slots, positions past the window
   dilated_swa         B=1 H=32 H_kv=8 N=32768 d=128, causal dilated window: 2048 taps
                       8 apart (receptive field 16384), blocks 128x64
+  topk_decode         64 sequences x 1 query, H=32 H_kv=8 d=128, cache length 131072,
+                      each query's 2048 highest-scoring keys (dynamic top-K)
 """
 from __future__ import annotations
 
@@ -91,6 +93,19 @@ class WindowDecodeWorkload:
     seed: int = 0
 
 
+@dataclass
+class TopkDecodeWorkload:
+    """Decode queries attending to their top_k keys by relevance score."""
+    name: str
+    S: int
+    H: int
+    H_kv: int
+    d: int
+    L: int
+    top_k: int
+    seed: int = 0
+
+
 WORKLOADS = {
     "tiny_static": PrefillWorkload("tiny_static", B=1, H=2, H_kv=2, N=256, d=64, causal=1,
                                    window=64, n_global=4, block_q=64, block_k=64, seed=1000),
@@ -105,6 +120,8 @@ WORKLOADS = {
                                     n_idx=2048, H_idx=32, seed=5000),
     "window_decode": WindowDecodeWorkload("window_decode", S=64, H=32, H_kv=8, d=128,
                                           window=4096, n_global=4, max_pos=131071, seed=6000),
+    "topk_decode": TopkDecodeWorkload("topk_decode", S=64, H=32, H_kv=8, d=128, L=131072,
+                                      top_k=2048, seed=8000),
     "dilated_swa": PrefillWorkload("dilated_swa", B=1, H=32, H_kv=8, N=32768, d=128, causal=1,
                                    window=2048, dilation=8, block_q=128, block_k=64, seed=7000),
 }
@@ -176,6 +193,15 @@ def _peaked(w: PrefillWorkload, Q, K, base: int, device):
 def calibration_inputs(w: PrefillWorkload, device="cpu"):
     """The calibration draw: same recipe, seed base + 100."""
     return prefill_inputs(w, device=device, seed=w.seed + 100)
+
+
+def topk_decode_inputs(w: TopkDecodeWorkload, device="cpu", seed: Optional[int] = None):
+    """(Q [S][H][d], K, V [S][H_kv][L][d]) -- N(0,1) draws, every key valid."""
+    base = w.seed if seed is None else seed
+    Q = randn_bf16((w.S, w.H, w.d), base, device)
+    K = randn_bf16((w.S, w.H_kv, w.L, w.d), base + 1, device)
+    V = randn_bf16((w.S, w.H_kv, w.L, w.d), base + 2, device)
+    return Q, K, V
 
 
 def gather_inputs(w: GatherWorkload, device="cpu", seed: Optional[int] = None):

@@ -9,7 +9,7 @@
  *   softmax(Q K^T / sqrt(d_k)) V ("sparse attention mechanism" glossary,
  *   chipfoundryservices, "Standard Attention Bottleneck").
  *
- * G_i comes from one of three places:
+ * G_i comes from one of four places:
  *   - sparse_attn_prefill*: a static pattern (sa_pattern_t) -- the union, by
  *     logical OR ("SAS: Sparse Attention Synthesizer", kindchill, Step 5,
  *     component 2), of a sliding window, global tokens, block-local blocks and
@@ -24,6 +24,8 @@
  *   - sparse_attn_gather: explicit index sets over a KV cache (decode).
  *   - sparse_attn_decode_window: the decode row of a causal window + global
  *     tokens pattern, over a cache of window + globals slots.
+ *   - sparse_attn_decode_topk: each decode query's top_k keys by relevance
+ *     score (a dynamic pattern, computed from the data at run time).
  *
  * K/V heads are shared by contiguous groups of query heads (GQA/MQA, glossary
  * "Multi-Query and Grouped-Query Attention"): h_kv = h / (H / H_kv).
@@ -247,6 +249,37 @@ int sparse_attn_decode_window(const void *Q, const void *K, const void *V,
                               const int32_t *positions, void *O, int S, int H, int H_kv,
                               int d, const sa_pattern_t *pat, float *lse_out,
                               sa_stream_t stream);
+
+/* Decode attention over the top_k keys of each query: the dynamic primitive
+ * "attend to the top-K dynamic tokens" ("SAS: Sparse Attention Synthesizer",
+ * Step 5, component 1, primitive C; the dynamic sparse patterns of "Sparse
+ * Attention Weights Assumption", whose G holds the tokens with the highest
+ * relevance scores).  For query (s, h) over the keys j < len_s of its K/V head:
+ * relevance s_j = scale * q . k_j (fp32), G = the k = min(top_k, len_s) keys
+ * with the largest s_j, equal scores to the smaller j; out = sum over G of
+ * softmax_G(s_j) v_j, lse = ln sum_G exp(s_j) (-inf and O = 0 for len_s = 0).
+ *   Q [S][H][d], K, V [S][H_kv][L][d] (bf16, device, read); O [S][H][d] (written).
+ *   lengths: device int32 [S] keys per sequence in [0, L], or NULL (all L);
+ *            a length outside [0, L] is clamped and recorded as SA_ERR_DEVICE_INDEX.
+ *   idx_out: device int32 [S][H][top_k] or NULL: the selected keys, ascending,
+ *            in the first idx_len entries (the rest untouched);
+ *   idx_len_out: device int32 [S][H] or NULL: k per query.
+ *   lse_out: device float [S][H] or NULL.
+ *   workspace: device memory of sparse_attn_decode_topk_workspace(S, H, L,
+ *            top_k) bytes, 16-byte aligned, owned by the caller, not read before
+ *            it is written; calls that overlap on the GPU need separate ones.
+ *   scale: 0 means 1/sqrt(d).
+ * Three kernels on `stream` (a score pass that reads every K row once per K/V
+ * head, an exact radix select, an attention pass over the selected V rows)
+ * plus a memset of the workspace histogram.  Errors: SA_ERR_INVALID_ARG
+ * (shapes, H % H_kv, top_k < 1, alignment, workspace too small),
+ * SA_ERR_UNSUPPORTED (d not 64/128, sizes past 32-bit grid limits). */
+size_t sparse_attn_decode_topk_workspace(int S, int H, int L, int top_k);
+int sparse_attn_decode_topk(const void *Q, const void *K, const void *V, const int32_t *lengths,
+                            void *O, int S, int H, int H_kv, int L, int d, int top_k,
+                            float scale, int32_t *idx_out, int32_t *idx_len_out,
+                            float *lse_out, void *workspace, size_t workspace_bytes,
+                            sa_stream_t stream);
 
 /* Cache slot of key j (j >= 0) in the layout of sparse_attn_decode_window;
  * -1 when j < 0, window < 1 or n_global < 0.  Host only. */
