@@ -242,12 +242,13 @@ static void row_attention(int kind, const void *Q, int64_t q_off,
                           const double *extra_s, int n_extra,
                           double *out, double *lse)
 {
-    if (nG == 0) {
+    if (nG == 0 && n_extra == 0) {
         for (int c = 0; c < d; ++c) out[c] = 0.0;
         *lse = -INFINITY;
         return;
     }
-    double *s = (double *)malloc(sizeof(double) * nG);
+    /* with nG == 0 but denominator-only terms, out = 0 and lse is theirs */
+    double *s = (double *)malloc(sizeof(double) * (size_t)(nG > 0 ? nG : 1));
     double m = -INFINITY;
     for (int k = 0; k < nG; ++k) {
         double acc = 0.0;

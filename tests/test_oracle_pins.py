@@ -448,3 +448,30 @@ def test_topk_sets_are_nested_and_exclude_the_rest(oracle_mod):
     V2[0, 0, out] += 100.0
     O2, _ = oracle_mod.gather(Q, K, V2, idx, n)
     assert np.max(np.abs(O1[0, 0] - O2[0, 0])) < 1e-14
+
+
+def test_bsfa_skipped_keys_in_denominator_variant(oracle_mod):
+    """The variant reading (skipped blocks' keys stay in the softmax
+    denominator): with every full block skipped (tau = +inf), lse is the dense
+    causal lse, and each row's output is the default-rule output scaled by
+    exp(lse_default - lse_variant) (same numerator, larger partition sum)."""
+    import torch
+    B, H, Hkv, N, d, Q, K, V = _bsfa_small(oracle_mod)
+    opat = oracle_mod.Pattern(causal=1)
+    tau = np.full(H, np.inf)
+    O0, l0 = oracle_mod.prefill(opat, Q, K, V, thresholds=tau)
+    O1, l1 = oracle_mod.prefill(opat, Q, K, V, thresholds=tau, keep_in_denominator=True)
+    s = torch.einsum("bhid,bjd->bhij", torch.from_numpy(Q), torch.from_numpy(K[:, 0])) / np.sqrt(d)
+    s = s.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), float("-inf"))
+    assert np.max(np.abs(torch.logsumexp(s, -1).numpy() - l1)) < 1e-10
+    assert np.max(np.abs(O0 * np.exp(l0 - l1)[..., None] - O1)) < 1e-12
+    # a tile whose blocks are all full and all skipped: O = 0, lse from the skipped keys alone
+    bl = oracle_mod.Pattern(causal=0, block_local=128)
+    Ob, lb = oracle_mod.prefill(bl, Q[:, :, :256], K[:, :, :256], V[:, :, :256], thresholds=tau,
+                                keep_in_denominator=True)
+    sb = torch.einsum("bhid,bjd->bhij", torch.from_numpy(Q[:, :, :256]),
+                      torch.from_numpy(K[:, 0, :256])) / np.sqrt(d)
+    blk = torch.arange(256) // 128
+    sb = sb.masked_fill(blk[:, None] != blk[None, :], float("-inf"))
+    assert np.all(Ob == 0)
+    assert np.max(np.abs(torch.logsumexp(sb, -1).numpy() - lb)) < 1e-10
