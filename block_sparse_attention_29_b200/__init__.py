@@ -48,6 +48,7 @@ class Pattern:
     random_table: Optional[np.ndarray] = None   # host int32 [H][ceil(N/rb)][n_random]
     scale: float = 0.0
     dilation: int = 1   # window taps this far apart (dilated/strided window); 1 = contiguous
+    skipped_in_denominator: int = 0   # block-skip variant: skipped keys stay in the denominator
 
     def to_c(self, thresholds_ptr: int = 0):
         tab = None
@@ -56,7 +57,8 @@ class Pattern:
         st = SaPattern(self.causal, self.window, self.n_global, self.block_local, self.block_q,
                        self.block_k, self.random_block, self.n_random if tab is not None else 0,
                        tab.ctypes.data if tab is not None else None,
-                       thresholds_ptr or None, self.scale, self.dilation)
+                       thresholds_ptr or None, self.scale, self.dilation,
+                       self.skipped_in_denominator)
         return st, tab   # the caller keeps `tab` alive while the struct is used
 
 

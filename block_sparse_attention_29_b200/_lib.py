@@ -39,7 +39,8 @@ class SaPattern(ctypes.Structure):
                 ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
                 ("random_block", ctypes.c_int32), ("n_random", ctypes.c_int32),
                 ("random_table", ctypes.c_void_p), ("thresholds", ctypes.c_void_p),
-                ("scale", ctypes.c_float), ("dilation", ctypes.c_int32)]
+                ("scale", ctypes.c_float), ("dilation", ctypes.c_int32),
+                ("skipped_in_denominator", ctypes.c_int32)]
 
 
 class SaPlanInfo(ctypes.Structure):

@@ -191,6 +191,7 @@ std::string cache_key(const sa_pattern_t* p, int B, int H, int Hkv, int N, int d
   auto put = [&k](const void* src, size_t n) { k.append(static_cast<const char*>(src), n); };
   const int32_t f[] = {p->causal, p->window, p->n_global, p->block_local, p->block_q,
                        p->block_k, p->random_block, p->n_random, p->dilation > 1 ? p->dilation : 1,
+                       p->skipped_in_denominator ? 1 : 0,
                        B, H, Hkv, N, d, dev};
   put(f, sizeof f);
   put(&p->scale, sizeof p->scale);
@@ -242,6 +243,7 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
   p->block_local = plan->pat.block_local;
   p->random_block = plan->pat.random_block;
   p->n_random = plan->d_rtab ? plan->pat.n_random : 0;
+  p->skip_denominator = plan->pat.skipped_in_denominator ? 1 : 0;
   const float scale = plan->pat.scale != 0.f ? plan->pat.scale : 1.0f / sqrtf(float(plan->d));
   p->scale = scale;
   p->scale_log2 = scale * 1.4426950408889634f;
@@ -294,10 +296,11 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
   rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
   if (rc) return rc;
   const int dil = pat->dilation > 1 ? pat->dilation : 1;
-  if (kernel == SA_KERNEL_PAIRED_HEADS && (dil > 1 || !pair_kernel_fits(d, H, H_kv, cp.H_pat)))
+  if (kernel == SA_KERNEL_PAIRED_HEADS &&
+      (dil > 1 || pat->skipped_in_denominator || !pair_kernel_fits(d, H, H_kv, cp.H_pat)))
     return set_error(SA_ERR_UNSUPPORTED,
                      "the paired-head kernel needs d = 128, an even number of query heads per "
-                     "K/V head, no random table and no dilation");
+                     "K/V head, no random table, no dilation and skipped keys out of G");
 
   sa_plan_t* plan = new sa_plan_t;
   plan->pat = *pat;
@@ -427,6 +430,7 @@ int sparse_attn_block_stats(const sa_plan_t* plan, const void* Q, const void* K,
   p.gate = 1;
   p.stats_only = 1;
   p.want_stats = 1;
+  p.skip_denominator = 0;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (block_mask_out) {
     cudaError_t e = cudaMemsetAsync(block_mask_out, 0,

@@ -59,6 +59,7 @@ struct PrefillParams {
   int pair;        // 1: units are head pairs (paired-head kernel), 0: single heads
   int gate;        // 1: statistics + decision per block (rule or stats pass)
   int stats_only;  // 1: no PV, no output (statistics pass)
+  int skip_denominator;  // 1: a skipped block's exp terms still enter m and l
   int want_stats;  // 1: block statistics needed (stat_out or gate)
   float scale;       // logit scale
   float scale_log2;  // scale * log2(e)

@@ -772,6 +772,8 @@ int launch_prefill_pair(const PrefillParams& p, int d, cudaStream_t stream) {
   if (p.head_pat || p.H % 2 || (p.H / p.Hkv) % 2)
     return set_error(SA_ERR_INVALID_ARG, "paired-head kernel: heads cannot be paired");
   if (p.dil != 1) return set_error(SA_ERR_UNSUPPORTED, "paired-head kernel: dilated window");
+  if (p.skip_denominator)
+    return set_error(SA_ERR_UNSUPPORTED, "paired-head kernel: skipped keys kept in the denominator");
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");

@@ -479,8 +479,13 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       }
       if (!keep) {
         if (leader) mbar_arrive_cnt(smem_u32(&bars->p_ready[fb]), kSoftmaxWarps);
-        ++g;
-        continue;
+        // Default rule: the block's keys leave G.  Variant: they stay in the
+        // denominator -- the max and the row sum below take them, no P is
+        // written (the S buffer is already handed back) and no PV runs.
+        if (!p.skip_denominator) {
+          ++g;
+          continue;
+        }
       }
 
       // Online softmax in the log2 domain with a lazily updated max.
@@ -533,6 +538,10 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         float s0, s1;
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
         l += s0 + s1;
+      }
+      if (!keep) {   // skipped, kept in the denominator only
+        ++g;
+        continue;
       }
       // P (bf16 pairs) over the first 32 columns of this block's S buffer,
       // whose logits are in registers.

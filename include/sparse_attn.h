@@ -110,6 +110,11 @@ typedef struct {
                                       thresholds per call.                                */
     float scale;
     int32_t dilation;              /* window taps k apart; 0 or 1 = contiguous window    */
+    int32_t skipped_in_denominator;/* block-skip rule variant: 1 keeps the keys of a
+                                      skipped block in the softmax denominator (no V
+                                      load and no PV for it, but its exp terms enter
+                                      l and the running max); 0 = they leave G_i.
+                                      Single-head kernel only.                          */
 } sa_pattern_t;
 
 /* A compiled pattern: per-(head, 128-row query tile) lists of 64-key blocks

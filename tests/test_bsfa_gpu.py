@@ -62,6 +62,47 @@ def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d, kernel):
     assert_close(lse, lr, what="lse")
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_bsfa_skipped_keys_in_denominator(product, oracle_mod, cuda, d):
+    """Variant rule: a skipped block's keys stay in the softmax denominator
+    (no V load, no PV).  Same mask comparison as the default rule; outputs and
+    lse against the oracle's variant reading."""
+    w = _small(d=d)
+    Qc, Kc, Vc, _ = calibration_inputs(w, device="cpu")
+    opat = oracle_mod.Pattern(**w.pattern_fields())
+    full_c, stat_c, _ = oracle_mod.block_stats(opat, Qc, Kc)
+    tau = oracle_mod.calibrate_thresholds(full_c, stat_c).astype(np.float32).astype(np.float64)
+    Q, K, V = _tensors(w, cuda)
+    pat = product.Pattern(**w.pattern_fields(), skipped_in_denominator=1)
+    plan = product.Plan(pat, w.B, w.H, w.H_kv, w.N, w.d)
+    tau_d = torch.tensor(tau, dtype=torch.float32, device=cuda)
+    mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
+    lse = torch.empty((w.B, w.H, w.N), device=cuda)
+    O = plan.prefill(Q, K, V, thresholds=tau_d, lse=lse, block_mask=mask)
+    lse0 = torch.empty_like(lse)
+    O0 = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N,
+                      w.d).prefill(Q, K, V, thresholds=tau_d, lse=lse0)
+    product.check_device_error()
+    Or, lr, om, ost, ofull = oracle_mod.prefill(opat, Q.cpu(), K.cpu(), V.cpu(), thresholds=tau,
+                                                keep_in_denominator=True, want_blocks=True)
+    n, n_near, override = compare_masks(mask.cpu().numpy(), om, ost, tau)
+    assert (om == 2).sum() > 0
+    if n_near:
+        Or, lr = oracle_mod.prefill(opat, Q.cpu(), K.cpu(), V.cpu(), thresholds=tau,
+                                    override=override, keep_in_denominator=True)
+    assert_close(O, Or)
+    assert_close(lse, lr, what="lse")
+    # the partition sum only grows: lse(variant) >= lse(default rule) on every row
+    assert torch.all(lse >= lse0 - 1e-4)
+
+
+def test_bsfa_denominator_variant_is_single_head_only(product, cuda):
+    w = _small()
+    with pytest.raises(product.SparseAttnError):
+        product.Plan(product.Pattern(**w.pattern_fields(), skipped_in_denominator=1), w.B, w.H,
+                     w.H_kv, w.N, w.d, kernel=product.KERNEL_PAIRED_HEADS)
+
+
 @pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
 def test_bsfa_extreme_thresholds(product, oracle_mod, cuda, kernel):
     w = _small(N=768, H=2, Hkv=1)
