@@ -6,7 +6,9 @@
 One step = one pass of the hot path over one batch of synthetic input: for a
 prefill workload one sparse_attn_prefill_plan launch (pattern compile and, for
 the block-skip workload, the one-time threshold calibration happen before the
-timed region); for gather_decode one sparse_attn_gather launch.
+timed region); for gather_decode one sparse_attn_gather launch; for
+window_decode one sparse_attn_decode_window launch; for topk_decode one
+sparse_attn_decode_topk call (score, select and attend kernels).
 
 Timing: W untimed warm-up steps, then exactly K steps bracketed by a barrier
 and torch.cuda.synchronize() on both sides.  L2 is flushed (256 MiB write)
@@ -320,7 +322,9 @@ def setup_topk_decode(w, device, torch, sa, workloads):
                 dense_flops=flops, algo_bytes=algo_bytes,
                 extra={"k_bytes_scored": k_bytes, "v_bytes_selected": v_bytes,
                        "workspace_bytes": ws.numel()},
-                kernel="topk_score_kernel", kernel_files=["topk_sm100.cu"],
+                # the roofline unit is the whole step (score, select and attend
+                # kernels): its traffic is the three kernels' DRAM bytes together
+                kernel="topk_step", kernel_files=["topk_sm100.cu"],
                 launches_per_step=3,
                 metric="top-K decode GB/s", unit="GB/s", bound="hbm",
                 tensors=(Q, K, V, None, O))
@@ -452,6 +456,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sequences", type=int, default=0,
+                    help="decode workloads: run this many sequences instead of the workload's "
+                         "(a reduced case of the same kernels, e.g. for counter captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -460,6 +467,11 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     from block_sparse_attention_29_b200 import workloads
     w = workloads.WORKLOADS[args.workload]
+    if args.sequences > 0:
+        import dataclasses
+        if not hasattr(w, "S"):
+            raise SystemExit("--sequences applies to the decode workloads only")
+        w = dataclasses.replace(w, S=args.sequences)
 
     if args.impl == "reference":
         if rank != 0:

@@ -14,10 +14,12 @@
 //      of the top 11 bits of its order-preserving key, kept in shared memory
 //      and added to global memory once per CTA.
 //   2. select: one CTA per (sequence, head) -- an exact radix select: the
-//      histogram gives the 11-bit bin of the top_k-th largest key, two passes
-//      over the head's scores resolve the next 11 and the last 10 bits, and a
-//      last pass writes the selected indices in ascending order (block-wide
-//      prefix sums), taking equal keys in index order.
+//      histogram gives the 11-bit bin of the top_k-th largest key; one sweep
+//      over the head's scores keeps that bin's keys in shared memory (up to
+//      8192; more take a slower path of three sweeps) and counts, per warp
+//      segment of the row, the keys above it; the threshold's last 21 bits
+//      are resolved in shared memory; a second sweep writes the selected
+//      indices in ascending order, equal keys in index order.
 //   3. attend: one CTA per (sequence, head) -- online softmax over the stored
 //      scores of the selected keys and the weighted sum of their V rows.
 #include <cuda_bf16.h>
@@ -57,6 +59,11 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 __device__ __forceinline__ uint32_t topk_key(float x) {
   const uint32_t u = __float_as_uint(x == 0.f ? 0.f : x);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The float whose key is `key` (the inverse of topk_key).
+__device__ __forceinline__ float topk_key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
 // Keys of sequence s: lengths[s] clamped to [0, L] (an out-of-range length is
@@ -231,10 +238,144 @@ __device__ __forceinline__ void find_bin(const uint32_t* h, uint32_t r, uint32_t
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(const TopkParams p) {
-  __shared__ uint32_t h[kTopkBins1];
-  __shared__ uint32_t ws[33];
-  __shared__ int res[2];
+constexpr int kSelUnroll = 4;      // float4 loads in flight per thread in a sweep
+constexpr int kCandCap = 8192;     // keys of the threshold's first-level bin kept in shared memory
+constexpr int kSegs = kSelectThreads / 32;   // row segments: one per warp
+
+struct SelectSmem {
+  uint32_t h[kTopkBins1];
+  uint32_t cand_key[kCandCap];
+  int32_t cand_j[kCandCap];
+  uint32_t ws[33];
+  int res[2];
+  uint32_t n_cand;
+  uint32_t seg_sure[kSegs], seg_sel[kSegs], seg_tie[kSegs], seg_off[kSegs], tie_before[kSegs];
+};
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x;
+}
+
+// One sweep over the scores of a row, j in [0, len): f(j, key) for every key,
+// kSelUnroll float4 loads issued per thread before any is used.  Rows are
+// padded to a multiple of 4 floats, so a float4 that starts below len is in
+// bounds.
+template <class F>
+__device__ __forceinline__ void sweep(const float* sc, int len, F&& f) {
+  constexpr int STEP = kSelectThreads * 4;
+  for (int c0 = threadIdx.x * 4; c0 < len; c0 += STEP * kSelUnroll) {
+    float4 v[kSelUnroll];
+#pragma unroll
+    for (int u = 0; u < kSelUnroll; ++u) {
+      const int j0 = c0 + u * STEP;
+      v[u] = j0 < len ? *reinterpret_cast<const float4*>(sc + j0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kSelUnroll; ++u) {
+      const int j0 = c0 + u * STEP;
+      const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (j0 + i < len) f(j0 + i, topk_key(x[i]));
+    }
+  }
+}
+
+__device__ __forceinline__ void select_failed(const TopkParams& p, int sh, int site) {
+  if (threadIdx.x == 0) {
+    record_device_error(p.err, SA_ERR_DEVICE_INDEX, site);
+    p.idx_len[sh] = 0;
+  }
+}
+
+// Selection when the threshold's first-level bin holds more keys than shared
+// memory keeps: two more sweeps resolve bits 20..10 and 9..0 of the
+// threshold, and a last one ranks the keys chunk by chunk in index order with
+// block-wide prefix sums.
+__device__ __noinline__ void select_generic(const TopkParams& p, SelectSmem& sm, const float* sc,
+                                            int len, int k, int b1, uint32_t r1, int32_t* out,
+                                            int sh) {
+  uint32_t* h = sm.h;
+  for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads) h[i] = 0;
+  __syncthreads();
+  sweep(sc, len, [&](int, uint32_t key) {
+    if ((key >> 21) == uint32_t(b1)) atomicAdd(&h[(key >> 10) & 2047u], 1u);
+  });
+  __syncthreads();
+  find_bin<kTopkBins1>(h, r1, sm.ws, sm.res);
+  const int b2 = sm.res[0];
+  const uint32_t r2 = uint32_t(sm.res[1]);
+  __syncthreads();
+  const uint32_t pre = (uint32_t(b1) << 11) | uint32_t(b2 < 0 ? 0 : b2);
+  for (int i = threadIdx.x; i < 1024; i += kSelectThreads) h[i] = 0;
+  __syncthreads();
+  sweep(sc, len, [&](int, uint32_t key) {
+    if ((key >> 10) == pre) atomicAdd(&h[key & 1023u], 1u);
+  });
+  __syncthreads();
+  find_bin<1024>(h, r2, sm.ws, sm.res);
+  const int b3 = sm.res[0];
+  const uint32_t take_eq = uint32_t(sm.res[1]);
+  __syncthreads();
+  if (b2 < 0 || b3 < 0) return select_failed(p, sh, 5);
+  const uint32_t thr = (pre << 10) | uint32_t(b3);
+
+  constexpr int STEP = kSelectThreads * 4;
+  uint32_t n_out = 0, n_eq = 0;
+  for (int c0 = 0; c0 < len; c0 += STEP) {
+    const int j0 = c0 + threadIdx.x * 4;
+    const float4 f = j0 < len ? *reinterpret_cast<const float4*>(sc + j0)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float x[4] = {f.x, f.y, f.z, f.w};
+    bool gt[4], eq[4];
+    uint32_t ce = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t key = topk_key(x[i]);
+      const bool in = j0 + i < len;
+      gt[i] = in && key > thr;
+      eq[i] = in && key == thr;
+      ce += eq[i];
+    }
+    uint32_t eq_total;
+    uint32_t eq_rank = n_eq + block_excl_scan(ce, sm.ws, &eq_total);
+    bool sel[4];
+    uint32_t cs = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sel[i] = gt[i] || (eq[i] && eq_rank < take_eq);
+      eq_rank += eq[i];
+      cs += sel[i];
+    }
+    uint32_t sel_total;
+    uint32_t pos = n_out + block_excl_scan(cs, sm.ws, &sel_total);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (sel[i] && pos < uint32_t(k)) out[pos++] = j0 + i;
+    n_out += sel_total;
+    n_eq += eq_total;
+  }
+  if (threadIdx.x == 0) {
+    if (n_out != uint32_t(k)) record_device_error(p.err, SA_ERR_DEVICE_INDEX, 6);
+    p.idx_len[sh] = int(min(n_out, uint32_t(k)));
+  }
+}
+
+// Common case: the row is split into 32 contiguous segments, one per warp.
+// Sweep 1 counts, per segment, the keys above the threshold's first-level bin
+// and keeps the bin's keys (with their indices) in shared memory; the
+// threshold's last 21 bits are resolved there; a 32-entry prefix sum gives
+// each segment its first output position; sweep 2 writes each segment's
+// selected indices in order, ranked inside the warp by shuffles.
+__global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) unsigned char smraw[];
+  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smraw);
   const int sh = blockIdx.x;
   const int s = sh / p.H;
   const int len = seq_len(p, s, 4);
@@ -249,106 +390,169 @@ __global__ void __launch_bounds__(kSelectThreads) topk_select_kernel(const TopkP
 
   // level 1: top 11 bits, from the score pass's histogram
   for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads)
-    h[i] = p.hist[(int64_t)sh * kTopkBins1 + i];
+    sm.h[i] = p.hist[(int64_t)sh * kTopkBins1 + i];
   __syncthreads();
-  find_bin<kTopkBins1>(h, uint32_t(k), ws, res);
-  const int b1 = res[0];
-  const uint32_t r1 = uint32_t(res[1]);
+  find_bin<kTopkBins1>(sm.h, uint32_t(k), sm.ws, sm.res);
+  const int b1 = sm.res[0];
+  const uint32_t r1 = uint32_t(sm.res[1]);
+  const uint32_t c1 = b1 >= 0 ? sm.h[b1] : 0u;
+  // bins 0-3 and 2044-2047 hold the infinities and NaNs
+  const uint32_t n_special = sm.h[0] + sm.h[1] + sm.h[2] + sm.h[3] + sm.h[2044] + sm.h[2045] +
+                             sm.h[2046] + sm.h[2047];
   __syncthreads();
-  if (b1 < 0) {   // the histogram does not hold len keys: inconsistent workspace
-    if (threadIdx.x == 0) {
-      record_device_error(p.err, SA_ERR_DEVICE_INDEX, 5);
-      p.idx_len[sh] = 0;
-    }
-    return;
-  }
-  // level 2: bits 20..10 of the keys in bin b1
-  for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads) h[i] = 0;
-  __syncthreads();
-  for (int j0 = threadIdx.x * 4; j0 < len; j0 += kSelectThreads * 4) {
-    const float4 f = *reinterpret_cast<const float4*>(sc + j0);   // rows padded to Lp
-    const float x[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t key = topk_key(x[i]);
-      if (j0 + i < len && (key >> 21) == uint32_t(b1)) atomicAdd(&h[(key >> 10) & 2047u], 1u);
-    }
-  }
-  __syncthreads();
-  find_bin<kTopkBins1>(h, r1, ws, res);
-  const int b2 = res[0];
-  const uint32_t r2 = uint32_t(res[1]);
-  __syncthreads();
-  // level 3: bits 9..0 of the keys with prefix (b1, b2)
-  const uint32_t pre = (uint32_t(b1) << 11) | uint32_t(b2 < 0 ? 0 : b2);
-  for (int i = threadIdx.x; i < 1024; i += kSelectThreads) h[i] = 0;
-  __syncthreads();
-  for (int j0 = threadIdx.x * 4; j0 < len; j0 += kSelectThreads * 4) {
-    const float4 f = *reinterpret_cast<const float4*>(sc + j0);
-    const float x[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t key = topk_key(x[i]);
-      if (j0 + i < len && (key >> 10) == pre) atomicAdd(&h[key & 1023u], 1u);
-    }
-  }
-  __syncthreads();
-  find_bin<1024>(h, r2, ws, res);
-  const int b3 = res[0];
-  const uint32_t take_eq = uint32_t(res[1]);   // keys equal to the threshold to take
-  __syncthreads();
-  if (b2 < 0 || b3 < 0) {
-    if (threadIdx.x == 0) {
-      record_device_error(p.err, SA_ERR_DEVICE_INDEX, 5);
-      p.idx_len[sh] = 0;
-    }
-    return;
-  }
-  const uint32_t thr = (pre << 10) | uint32_t(b3);
+  if (b1 < 0) return select_failed(p, sh, 5);   // the histogram does not hold len keys
+  // The sweeps below compare the floats themselves with the bounds of bin b1
+  // and with the threshold (key order is float order, NaN aside); the bounds
+  // must be numbers, which holds for bins 4 .. 2043, and the row must hold no
+  // infinity or NaN (bins 0-3 and 2044-2047), which the key order ranks but
+  // float comparisons do not.
+  if (c1 > uint32_t(kCandCap) || b1 < 4 || b1 > 2043 || n_special != 0)
+    return select_generic(p, sm, sc, len, k, b1, r1, out, sh);
+  const float f_lo = topk_key_float(uint32_t(b1) << 21);        // x >= f_lo: bin >= b1
+  const float f_hi = topk_key_float(uint32_t(b1 + 1) << 21);    // x >= f_hi: bin >  b1
 
-  // output: keys above the threshold and the first take_eq equal ones, in
-  // ascending index order
-  uint32_t n_out = 0, n_eq = 0;
-  for (int c0 = 0; c0 < len; c0 += kSelectThreads * 4) {
-    const int j0 = c0 + threadIdx.x * 4;
-    bool gt[4], eq[4];
-    uint32_t ce = 0;
-    if (j0 < len) {
-      const float4 f = *reinterpret_cast<const float4*>(sc + j0);
-      const float x[4] = {f.x, f.y, f.z, f.w};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = (((len + kSegs - 1) / kSegs) + 127) & ~127;   // a multiple of 128 keys
+  const int lo = warp * seg, hi = min(len, lo + seg);
+  if (threadIdx.x == 0) sm.n_cand = 0;
+  if (threadIdx.x < kSegs) sm.seg_sel[threadIdx.x] = sm.seg_tie[threadIdx.x] = 0;
+  __syncthreads();
+
+  // sweep 1
+  uint32_t sure = 0;
+  for (int c0 = lo + lane * 4; c0 < hi; c0 += 128 * kSelUnroll) {
+    float4 v[kSelUnroll];
+#pragma unroll
+    for (int u = 0; u < kSelUnroll; ++u) {
+      const int j0 = c0 + u * 128;
+      v[u] = j0 < hi ? *reinterpret_cast<const float4*>(sc + j0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kSelUnroll; ++u) {
+      const int j0 = c0 + u * 128;
+      const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      // most scores lie below the bin: one test per float4 skips them
+      if (!(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])) >= f_lo)) continue;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t key = topk_key(x[i]);
-        const bool in = j0 + i < len;
-        gt[i] = in && key > thr;
-        eq[i] = in && key == thr;
-        ce += eq[i];
+        if (j0 + i < hi) {
+          if (x[i] >= f_hi) {
+            ++sure;
+          } else if (x[i] >= f_lo) {
+            const uint32_t slot = atomicAdd(&sm.n_cand, 1u);
+            if (slot < uint32_t(kCandCap)) {
+              sm.cand_key[slot] = topk_key(x[i]);
+              sm.cand_j[slot] = j0 + i;
+            }
+          }
+        }
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) gt[i] = eq[i] = false;
     }
-    uint32_t eq_total;
-    uint32_t eq_rank = n_eq + block_excl_scan(ce, ws, &eq_total);
-    bool sel[4];
-    uint32_t cs = 0;
+  }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      sel[i] = gt[i] || (eq[i] && eq_rank < take_eq);
-      eq_rank += eq[i];
-      cs += sel[i];
+  for (int o = 16; o > 0; o >>= 1) sure += __shfl_xor_sync(0xffffffffu, sure, o);
+  if (lane == 0) sm.seg_sure[warp] = sure;
+  for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads) sm.h[i] = 0;
+  __syncthreads();
+  const uint32_t nc = min(sm.n_cand, uint32_t(kCandCap));   // == c1
+
+  // level 2 and level 3 over the kept keys
+  for (uint32_t c = threadIdx.x; c < nc; c += kSelectThreads)
+    atomicAdd(&sm.h[(sm.cand_key[c] >> 10) & 2047u], 1u);
+  __syncthreads();
+  find_bin<kTopkBins1>(sm.h, r1, sm.ws, sm.res);
+  const int b2 = sm.res[0];
+  const uint32_t r2 = uint32_t(sm.res[1]);
+  __syncthreads();
+  const uint32_t pre = (uint32_t(b1) << 11) | uint32_t(b2 < 0 ? 0 : b2);
+  for (int i = threadIdx.x; i < 1024; i += kSelectThreads) sm.h[i] = 0;
+  __syncthreads();
+  for (uint32_t c = threadIdx.x; c < nc; c += kSelectThreads) {
+    const uint32_t key = sm.cand_key[c];
+    if ((key >> 10) == pre) atomicAdd(&sm.h[key & 1023u], 1u);
+  }
+  __syncthreads();
+  find_bin<1024>(sm.h, r2, sm.ws, sm.res);
+  const int b3 = sm.res[0];
+  const uint32_t take_eq = uint32_t(sm.res[1]);   // keys equal to the threshold to take
+  __syncthreads();
+  if (b2 < 0 || b3 < 0 || nc != c1) return select_failed(p, sh, 5);
+  const uint32_t thr = (pre << 10) | uint32_t(b3);
+  const float f_thr = topk_key_float(thr);   // a score of the row, so a number
+
+  // kept keys above the threshold and keys equal to it, per segment
+  for (uint32_t c = threadIdx.x; c < nc; c += kSelectThreads) {
+    const uint32_t key = sm.cand_key[c];
+    const int sg = sm.cand_j[c] / seg;
+    if (key > thr) atomicAdd(&sm.seg_sel[sg], 1u);
+    else if (key == thr) atomicAdd(&sm.seg_tie[sg], 1u);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // equal keys are taken in index order: the first take_eq of them
+    const uint32_t tie = sm.seg_tie[lane];
+    const uint32_t tie_before = warp_incl_scan(tie) - tie;
+    const uint32_t taken = take_eq > tie_before ? min(tie, take_eq - tie_before) : 0u;
+    const uint32_t tot = sm.seg_sure[lane] + sm.seg_sel[lane] + taken;
+    const uint32_t incl = warp_incl_scan(tot);
+    sm.seg_off[lane] = incl - tot;
+    sm.tie_before[lane] = tie_before;
+    if (lane == 31) sm.res[0] = int(incl);
+  }
+  __syncthreads();
+
+  // sweep 2: the selected indices of each segment, in order
+  uint32_t run = sm.seg_off[warp];
+  uint32_t tie_run = sm.tie_before[warp];
+  for (int c0 = lo; c0 < hi; c0 += 128 * kSelUnroll) {
+    float4 v[kSelUnroll];
+#pragma unroll
+    for (int u = 0; u < kSelUnroll; ++u) {
+      const int j0 = c0 + u * 128 + lane * 4;
+      v[u] = j0 < hi ? *reinterpret_cast<const float4*>(sc + j0) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    uint32_t sel_total;
-    uint32_t pos = n_out + block_excl_scan(cs, ws, &sel_total);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (sel[i] && pos < uint32_t(k)) out[pos++] = j0 + i;
-    n_out += sel_total;
-    n_eq += eq_total;
+    for (int u = 0; u < kSelUnroll; ++u) {
+      if (c0 + u * 128 >= hi) break;   // the same for the whole warp
+      const int j0 = c0 + u * 128 + lane * 4;
+      const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      bool gt[4] = {false, false, false, false}, eq[4] = {false, false, false, false};
+      uint32_t ct = 0;
+      if (fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])) >= f_thr) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const bool in = j0 + i < hi;
+          gt[i] = in && x[i] > f_thr;
+          eq[i] = in && x[i] == f_thr;
+          ct += eq[i];
+        }
+      }
+      uint32_t tr = tie_run;
+      if (__any_sync(0xffffffffu, ct != 0)) {
+        const uint32_t incl = warp_incl_scan(ct);
+        tr += incl - ct;
+        tie_run += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      bool sel[4];
+      uint32_t cs = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sel[i] = gt[i] || (eq[i] && tr < take_eq);
+        tr += eq[i];
+        cs += sel[i];
+      }
+      const uint32_t incl = warp_incl_scan(cs);
+      uint32_t pos = run + incl - cs;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (sel[i] && pos < uint32_t(k)) out[pos++] = j0 + i;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
   if (threadIdx.x == 0) {
-    if (n_out != uint32_t(k)) record_device_error(p.err, SA_ERR_DEVICE_INDEX, 6);
-    p.idx_len[sh] = int(min(n_out, uint32_t(k)));
+    const uint32_t total = uint32_t(sm.res[0]);
+    if (total != uint32_t(k)) record_device_error(p.err, SA_ERR_DEVICE_INDEX, 6);
+    p.idx_len[sh] = int(min(total, uint32_t(k)));
   }
 }
 
@@ -467,7 +671,10 @@ int launch_topk(const TopkParams& p, int d, cudaStream_t stream) {
   if (d == 128) { SA_SCORE(128) } else { SA_SCORE(64) }
 #undef SA_SCORE
   if (rc) return rc;
-  topk_select_kernel<<<(unsigned)n, kSelectThreads, 0, stream>>>(p);
+  const int sel_smem = int(sizeof(SelectSmem));
+  e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
+  if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute(top-k select)");
+  topk_select_kernel<<<(unsigned)n, kSelectThreads, sel_smem, stream>>>(p);
   if (d == 128) topk_attend_kernel<128><<<(unsigned)n, kAttendThreads, 0, stream>>>(p);
   else topk_attend_kernel<64><<<(unsigned)n, kAttendThreads, 0, stream>>>(p);
   e = cudaGetLastError();
