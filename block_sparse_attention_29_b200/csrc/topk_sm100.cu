@@ -373,7 +373,7 @@ __device__ __noinline__ void select_generic(const TopkParams& p, SelectSmem& sm,
 // threshold's last 21 bits are resolved there; a 32-entry prefix sum gives
 // each segment its first output position; sweep 2 writes each segment's
 // selected indices in order, ranked inside the warp by shuffles.
-__global__ void __launch_bounds__(kSelectThreads, 2) topk_select_kernel(const TopkParams p) {
+__global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const TopkParams p) {
   extern __shared__ __align__(16) unsigned char smraw[];
   SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smraw);
   const int sh = blockIdx.x;
