@@ -115,3 +115,65 @@ def test_struct_layouts_match_the_header(product, tmp_path):
         assert got[(cname, "size")] == ctypes.sizeof(py), cname
         for f, _ in py._fields_:
             assert got[(cname, f)] == getattr(py, f).offset, (cname, f)
+
+
+def test_decode_entry_points_reject_bad_arguments_on_host(product):
+    """Top-K and window decode: argument errors are found before any launch,
+    and the workspace size is the documented layout."""
+    L = product._lib.lib()
+    S, H, Lk, k = 3, 4, 1001, 50
+
+    def r256(n):
+        return (n + 255) // 256 * 256
+    Lp = (Lk + 3) // 4 * 4
+    want = r256(S * H * Lp * 4) + r256(S * H * 2048 * 4) + r256(S * H * k * 4) + r256(S * H * 4)
+    assert product.decode_topk_workspace_bytes(S, H, Lk, k) == want
+    assert product.decode_topk_workspace_bytes(S, H, Lk, 0) == 0
+
+    def topk(**kw):
+        a = dict(Q=16, K=16, V=16, lengths=None, O=16, S=S, H=H, Hkv=2, L=Lk, d=128, top_k=k,
+                 scale=0.0, idx=None, n=None, lse=None, ws=16, ws_bytes=want)
+        a.update(kw)
+        return _err(product, L.sparse_attn_decode_topk(
+            a["Q"], a["K"], a["V"], a["lengths"], a["O"], a["S"], a["H"], a["Hkv"], a["L"],
+            a["d"], a["top_k"], a["scale"], a["idx"], a["n"], a["lse"], a["ws"], a["ws_bytes"],
+            None))
+    assert topk(top_k=0)[0] == product.SA_ERR_INVALID_ARG
+    assert topk(Hkv=3)[0] == product.SA_ERR_INVALID_ARG
+    assert topk(d=96)[0] == product.SA_ERR_UNSUPPORTED
+    rc, msg = topk(ws_bytes=want - 1)
+    assert rc == product.SA_ERR_INVALID_ARG and "workspace" in msg
+    rc, msg = topk(ws=24)
+    assert rc == product.SA_ERR_INVALID_ARG and "aligned" in msg
+    assert topk(O=None)[0] == product.SA_ERR_INVALID_ARG
+
+    def window(**kw):
+        fields = dict(causal=1, window=64, n_global=2)
+        fields.update(kw)
+        pat, _t = product.Pattern(**fields).to_c()
+        return _err(product, L.sparse_attn_decode_window(16, 16, 16, 16, 16, 2, 4, 2, 128,
+                                                         ctypes.byref(pat), None, None))[0]
+    assert window(causal=0) == product.SA_ERR_UNSUPPORTED
+    assert window(window=0) == product.SA_ERR_UNSUPPORTED
+    assert window(dilation=2) == product.SA_ERR_UNSUPPORTED
+    assert window(block_local=64) == product.SA_ERR_UNSUPPORTED
+
+
+def test_plan_refusals_on_host(product):
+    """Combinations the kernels do not run are refused when the plan is made,
+    before any device allocation."""
+    L = product._lib.lib()
+    h = ctypes.c_void_p()
+
+    def plan(kernel=product.KERNEL_AUTO, N=600, H=4, Hkv=2, d=128, **fields):
+        pat, _t = product.Pattern(**fields).to_c()
+        return _err(product, L.sparse_attn_plan_create_ex(ctypes.byref(pat), 1, H, Hkv, N, d,
+                                                          kernel, ctypes.byref(h)))[0]
+    assert plan(causal=1, window=8, dilation=7) == product.SA_ERR_UNSUPPORTED      # 7 does not divide 600
+    assert plan(causal=1, window=8, dilation=3, n_global=2) == product.SA_ERR_UNSUPPORTED
+    assert plan(causal=1, window=0, dilation=3) == product.SA_ERR_INVALID_ARG
+    assert plan(causal=1, window=8, dilation=3,
+                kernel=product.KERNEL_PAIRED_HEADS) == product.SA_ERR_UNSUPPORTED
+    assert plan(causal=1, skipped_in_denominator=1,
+                kernel=product.KERNEL_PAIRED_HEADS) == product.SA_ERR_UNSUPPORTED
+    assert plan(causal=1, kernel=7) == product.SA_ERR_INVALID_ARG
