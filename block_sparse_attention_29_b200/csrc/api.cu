@@ -606,7 +606,9 @@ int sparse_attn_decode_topk(const void* Q, const void* K, const void* V, const i
   if (H % H_kv != 0) return set_error(SA_ERR_INVALID_ARG, "H = %d is not a multiple of H_kv = %d", H, H_kv);
   if (top_k < 1) return set_error(SA_ERR_INVALID_ARG, "top_k = %d (must be >= 1)", top_k);
   if (d != 64 && d != 128) return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
-  if (int64_t(S) * H > INT32_MAX || L > (1 << 29))
+  // grids: (S*H) CTAs in x for the select and attention passes; the score pass
+  // puts its 8192-key chunks in y (at most 65535 of them)
+  if (int64_t(S) * H > INT32_MAX || int64_t(L) > int64_t(65535) * kTopkChunk)
     return set_error(SA_ERR_UNSUPPORTED, "S*H or L too large for the launch grids");
   TopkLayout t;
   topk_layout(S, H, L, top_k, &t);

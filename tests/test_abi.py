@@ -146,6 +146,10 @@ def test_decode_entry_points_reject_bad_arguments_on_host(product):
     rc, msg = topk(ws=24)
     assert rc == product.SA_ERR_INVALID_ARG and "aligned" in msg
     assert topk(O=None)[0] == product.SA_ERR_INVALID_ARG
+    # more 8192-key chunks than a grid dimension holds
+    big = 65535 * 8192 + 1
+    assert topk(L=big, S=1, H=2, ws_bytes=product.decode_topk_workspace_bytes(1, 2, big, k))[0] == \
+        product.SA_ERR_UNSUPPORTED
 
     def window(**kw):
         fields = dict(causal=1, window=64, n_global=2)
