@@ -163,3 +163,35 @@ def test_topk_decode_full_size_sampled(product, oracle_mod, cuda):
         Or, lr = oracle_mod.gather(Qs, Ks, Vs, gi, gn)
         assert_close(O[s, h][None, None], Or)
         assert_close(lse[s, h].reshape(1, 1), lr, what="lse")
+
+
+@pytest.mark.parametrize("L,top_k,two_levels", [(4096, 300, False), (20000, 100, False),
+                                                 (20000, 12000, True)],
+                         ids=["ties-over-segments", "overfull-bin", "overfull-bin-two-levels"])
+def test_topk_decode_ties_in_index_order(product, oracle_mod, cuda, L, top_k, two_levels):
+    """Equal scores are taken in index order when they span several of the
+    select pass's row segments, and when the threshold's first-level bin holds
+    more keys than shared memory keeps (its three-sweep path).  Checked exactly:
+    the near-cut tolerance of the other tests would accept any choice of ties."""
+    S, H, Hkv, d = 1, 2, 1, 128
+    Q = _rand((S, H, d), L + top_k, cuda)
+    Q[0, 1] = Q[0, 0]
+    K = _rand((S, Hkv, L, d), L + top_k + 1, cuda)
+    V = _rand((S, Hkv, L, d), L + top_k + 2, cuda)
+    row_b = K[0, 0, 5].clone()
+    K[0, 0] = row_b
+    if two_levels:
+        # even keys score higher (the same row plus the query direction)
+        row_a = (row_b.float() + Q[0, 0].float() / Q[0, 0].float().norm()).to(torch.bfloat16)
+        K[0, 0, 0::2] = row_a
+        want = np.sort(np.concatenate([np.arange(0, L, 2), np.arange(1, L, 2)[:top_k - L // 2]]))
+    else:
+        want = np.arange(top_k)
+    O, idx, n = product.sparse_attn_decode_topk(Q, K, V, top_k)
+    product.check_device_error()
+    idx, n = idx.cpu().numpy(), n.cpu().numpy()
+    for h in range(H):
+        assert n[0, h] == top_k
+        assert np.array_equal(idx[0, h], want)
+    Or, _ = oracle_mod.gather(Q.cpu(), K.cpu(), V.cpu(), idx, n)
+    assert_close(O, Or)
