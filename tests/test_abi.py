@@ -181,3 +181,57 @@ def test_plan_refusals_on_host(product):
     assert plan(causal=1, skipped_in_denominator=1,
                 kernel=product.KERNEL_PAIRED_HEADS) == product.SA_ERR_UNSUPPORTED
     assert plan(causal=1, kernel=7) == product.SA_ERR_INVALID_ARG
+
+
+def test_c_program_uses_the_abi(product, tmp_path):
+    """A plain C program built against include/sparse_attn.h and linked to the
+    library calls its host-only entry points (pattern compiler, workspace size,
+    cache slot, error reporting) with the results the binding gets."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <stdlib.h>
+#include "sparse_attn.h"
+int main(void) {
+    sa_pattern_t p = {0};
+    p.causal = 1; p.window = 300; p.n_global = 4; p.block_q = 128; p.block_k = 64;
+    int H_pat = 0, T = 0; int64_t n = 0;
+    if (sparse_attn_compile_pattern(&p, 2, 1000, 128, 64, &H_pat, &T, &n, NULL, NULL, NULL, NULL))
+        return 1;
+    int32_t *row = malloc(sizeof(int32_t) * (H_pat * T + 1));
+    int32_t *kb = malloc(sizeof(int32_t) * n);
+    uint8_t *full = malloc(n);
+    int64_t *cnt = malloc(sizeof(int64_t) * n);
+    if (sparse_attn_compile_pattern(&p, 2, 1000, 128, 64, &H_pat, &T, &n, row, kb, full, cnt))
+        return 2;
+    long long pairs = 0, nfull = 0;
+    for (int64_t e = 0; e < n; ++e) { pairs += cnt[e]; nfull += full[e]; }
+    printf("%d %d %lld %lld %lld\n", H_pat, T, (long long)n, nfull, pairs);
+    printf("%zu\n", sparse_attn_decode_topk_workspace(3, 4, 1001, 50));
+    printf("%lld\n", (long long)sparse_attn_window_slot(5000, 4096, 4));
+    p.dilation = 7;
+    int rc = sparse_attn_compile_pattern(&p, 2, 1000, 128, 64, &H_pat, &T, &n, NULL, NULL, NULL, NULL);
+    printf("%d %s\n", rc, rc ? "refused" : "accepted");
+    printf("%d\n", sparse_attn_last_error()[0] != 0);
+    return 0;
+}
+''')
+    exe = tmp_path / "use_abi"
+    libdir = os.path.dirname(product.LIB_PATH)
+    libname = os.path.basename(product.LIB_PATH)[3:-3]
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, f"-l{libname}", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    row_ptr, kb, full, cnt, H_pat, T = product.compile_pattern(
+        product.Pattern(causal=1, window=300, n_global=4), 2, 1000)
+    assert out[0].split() == [str(H_pat), str(T), str(len(kb)), str(int(full.sum())),
+                              str(int(cnt.sum()))]
+    assert int(out[1]) == product.decode_topk_workspace_bytes(3, 4, 1001, 50)
+    assert int(out[2]) == product.window_slot(5000, 4096, 4) == 4 + 5000 % 4096
+    assert out[3].split() == [str(product.SA_ERR_UNSUPPORTED), "refused"]
+    assert out[4] == "1"
