@@ -31,13 +31,7 @@
 // 32 columns of that buffer once the logits are in registers, and the PV of
 // block k reads it there.  The QK^T of block k+1 runs while the softmax works
 // on block k, also when block k is skipped by the rule, so a run of skipped
-// blocks costs the softmax's statistic alone per block (with the variant
-// that keeps skipped keys in the denominator, also their exponentials).
-//
-// Dilated windows (taps k apart): a work unit is also indexed by its residue
-// class r; the tensor maps view [N][d] as [N/k][k][d], so the tiles of class r
-// are loaded as one TMA box each, and position m of the class is output row
-// m*k + r.
+// blocks costs the softmax's statistic alone per block.
 #include <cuda_bf16.h>
 
 #include <cmath>
