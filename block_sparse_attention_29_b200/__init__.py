@@ -10,10 +10,26 @@ Entry points mirror include/sparse_attn.h:
 * ``Plan`` -- sparse_attn_plan_create / _info / _destroy, ``Plan.prefill``
   (sparse_attn_prefill_plan), ``Plan.block_stats`` (sparse_attn_block_stats),
   ``Plan.calibrate`` (sparse_attn_calibrate).
-* ``sparse_attn_prefill`` -- one-shot prefill through the library's plan cache.
+* ``sparse_attn_prefill`` -- one-shot prefill through the library's plan cache;
+  ``sparse_attn_prefill_noalloc`` -- the same without device allocation.
 * ``sparse_attn_gather`` -- explicit index sets over a KV cache.
+* ``sparse_attn_decode_window`` / ``window_slot`` -- decode of a causal window +
+  global tokens pattern over a cache of window + globals slots.
+* ``sparse_attn_decode_topk`` / ``decode_topk_workspace_bytes`` -- decode over
+  each query's top_k keys by relevance score.
 * ``compile_pattern`` -- the host pattern compiler (no GPU needed).
 * ``check_device_error`` -- reads and clears the device error word.
+
+Example (a causal sliding window of 4096 with GQA, then the block-skip rule
+with thresholds calibrated on a calibration draw)::
+
+    import block_sparse_attention_29_b200 as sa
+    pat = sa.Pattern(causal=1, window=4096)            # block_q=128, block_k=64
+    plan = sa.Plan(pat, B, H, H_kv, N, d)              # compiled once, reusable
+    O = plan.prefill(Q, K, V)                          # bf16 [B][H][N][d]
+    rule = sa.Plan(sa.Pattern(causal=1), B, H, H_kv, N, d)
+    tau = rule.calibrate(rule.block_stats(Qc, Kc), 0.5)   # per-head thresholds
+    O = rule.prefill(Q, K, V, thresholds=tau)
 """
 from __future__ import annotations
 
