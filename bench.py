@@ -174,13 +174,16 @@ def prefill_accounting(w, info, kept_desc=None, skipped_pairs=0):
 
 def setup_prefill(w, device, torch, sa, workloads):
     Q, K, V, tab = workloads.prefill_inputs(w, device=device)
-    pat = sa.Pattern(**w.pattern_fields(), random_table=tab)
+    pat = sa.Pattern(**w.pattern_fields(), random_table=tab,
+                     skipped_in_denominator=w.skipped_in_denominator)
     plan = sa.Plan(pat, w.B, w.H, w.H_kv, w.N, w.d)
     thresholds = None
     extra = {"plan_compile_ms": round(plan.info["compile_ms"], 2)}
     kept_desc, skipped_pairs = None, 0
     if w.bsfa:
         Qc, Kc, _, _ = workloads.calibration_inputs(w, device=device)
+        # the statistics pass is the same for the denominator variant (it
+        # changes what a skipped block contributes, not the decision)
         thresholds = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
         del Qc, Kc
         mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=device)
@@ -435,7 +438,8 @@ def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
         rows = np.array([(b, h, m * k + r) for b, h, t, r in tiles
                          for m in range(t * 128, min(n_pos, t * 128 + 128))], np.int32)
         t0 = time.perf_counter()
-        oracle.prefill(opat, Qh, Kh, Vh, thresholds=thresholds, rows=rows, nthreads=cores)
+        oracle.prefill(opat, Qh, Kh, Vh, thresholds=thresholds, rows=rows, nthreads=cores,
+                       keep_in_denominator=bool(w.skipped_in_denominator))
         t_total += time.perf_counter() - t0
         for b, h, t, _r in tiles:
             hp = h if H_pat > 1 else 0
@@ -621,6 +625,7 @@ def config_of(w, world):
     pat = {k: v for k, v in w.pattern_fields().items() if v and not (k == "dilation" and v == 1)}
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
             "pattern": pat, "block_skip_rule": bool(w.bsfa),
+            **({"skipped_keys_in_denominator": True} if w.skipped_in_denominator else {}),
             "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}
 
 

@@ -25,6 +25,8 @@ Workloads (names used by tests and bench):
                       8 apart (receptive field 16384), blocks 128x64
   topk_decode         64 sequences x 1 query, H=32 H_kv=8 d=128, cache length 131072,
                       each query's 2048 highest-scoring keys (dynamic top-K)
+  bsfa_denominator    bsfa_causal's inputs and thresholds with the rule's variant that
+                      keeps skipped blocks' keys in the softmax denominator
 """
 from __future__ import annotations
 
@@ -54,6 +56,7 @@ class PrefillWorkload:
     bsfa: bool = False
     seed: int = 0
     dilation: int = 1
+    skipped_in_denominator: int = 0   # block-skip variant (product pattern field)
     extra: dict = field(default_factory=dict)
 
     def pattern_fields(self):
@@ -122,6 +125,9 @@ WORKLOADS = {
                                           window=4096, n_global=4, max_pos=131071, seed=6000),
     "topk_decode": TopkDecodeWorkload("topk_decode", S=64, H=32, H_kv=8, d=128, L=131072,
                                       top_k=2048, seed=8000),
+    "bsfa_denominator": PrefillWorkload("bsfa_denominator", B=1, H=32, H_kv=8, N=32768, d=128,
+                                        causal=1, block_q=128, block_k=64, bsfa=True,
+                                        skipped_in_denominator=1, seed=3000),
     "dilated_swa": PrefillWorkload("dilated_swa", B=1, H=32, H_kv=8, N=32768, d=128, causal=1,
                                    window=2048, dilation=8, block_q=128, block_k=64, seed=7000),
 }
