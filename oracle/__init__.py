@@ -76,7 +76,7 @@ def _load():
         lib.ora_tile_blocks.argtypes = [P, i32, i32, i32, i32, i32, i32, dbl, vp, vp,
                                         i32, i32, i32, vp, vp, vp, vp, vp, vp]
         lib.ora_prefill.argtypes = [P, i32, i32, i32, i32, i32, i32, dbl, vp, vp, vp,
-                                    vp, vp, i32, i64, vp, vp, vp, vp, vp, vp, i32]
+                                    vp, vp, i32, i32, vp, vp, i64, vp, vp, vp, vp, vp, vp, i32]
         lib.ora_dense.argtypes = [i32, i32, i32, i32, i32, i32, dbl, i32, vp, vp, vp, vp]
         lib.ora_gather.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, dbl, vp, vp, vp,
                                    vp, vp, vp, vp, i32]
@@ -214,14 +214,22 @@ def tile_blocks(p: Pattern, Q, K, b: int, h: int, t: int, thresholds=None, scale
 
 
 def prefill(p: Pattern, Q, K, V, thresholds=None, scale=None, rows=None, override=None,
-            keep_in_denominator=False, want_blocks=False, nthreads=0):
+            keep_in_denominator=False, want_blocks=False, nthreads=0, row_level=False,
+            row_override=None, want_row_stats=False):
     """Sparse attention prefill over static G_i, optionally with the block-skip rule.
 
     Q: [B][H][N][d]; K, V: [B][H_kv][N][d] (bf16 tensors or float64 arrays).
     rows: None (every row; returns O [B][H][N][d]) or int array [n][3] of
     (b, h, i) (returns O [n][d]).  Returns (O, lse) or, with want_blocks,
-    (O, lse, mask, stat) with mask/stat shaped [B][H][T][n_kb] (only tiles that
-    hold a requested row are filled).
+    (O, lse, mask, stat, full) with mask/stat/full shaped [B][H][T][n_kb] (only
+    tiles that hold a requested row are filled).
+
+    row_level: the per-query reading of the rule ("Block Sparse Flash
+    Attention", paper summary): each row also drops the full blocks of its
+    tile whose maximum over its own logits is below the threshold.
+    row_override: int8 [n_rows][n_kb] (-1 rule, 0 keep, 1 drop) for the
+    requested rows.  want_row_stats appends the rows' per-block maxima
+    ([n_rows][n_kb], -inf for blocks that are not full) to the result.
     """
     kq, q = _as_input(Q)
     kk, k = _as_input(K)
@@ -240,6 +248,12 @@ def prefill(p: Pattern, Q, K, V, thresholds=None, scale=None, rows=None, overrid
         n = B * H * N
     O = np.zeros((n, d), np.float64)
     lse = np.zeros(n, np.float64)
+    if row_level and keep_in_denominator:
+        raise ValueError("the row-level reading is not combined with keep_in_denominator")
+    rov = None if row_override is None else np.ascontiguousarray(row_override, np.int8)
+    if rov is not None:
+        assert row_level and rov.shape == (n, n_kb), (rov.shape, (n, n_kb))
+    rstat = np.full((n, n_kb), -np.inf) if want_row_stats else None
     th = None if thresholds is None else np.ascontiguousarray(thresholds, np.float64)
     ov = None if override is None else np.ascontiguousarray(override, np.int8)
     mask = stat = full = None
@@ -251,14 +265,18 @@ def prefill(p: Pattern, Q, K, V, thresholds=None, scale=None, rows=None, overrid
     _load().ora_prefill(ctypes.byref(st), kq, B, H, Hkv, N, d,
                         default_scale(d) if scale is None else scale,
                         q.ctypes.data, k.ctypes.data, v.ctypes.data, _p(th), _p(ov),
-                        1 if keep_in_denominator else 0, n, _p(r), O.ctypes.data,
+                        1 if keep_in_denominator else 0, 1 if row_level else 0, _p(rov),
+                        _p(rstat), n, _p(r), O.ctypes.data,
                         lse.ctypes.data, _p(mask), _p(stat), _p(full), nthreads)
     if rows is None:
         O = O.reshape(B, H, N, d)
         lse = lse.reshape(B, H, N)
+    res = (O, lse)
     if want_blocks:
-        return O, lse, mask, stat, full.astype(bool)
-    return O, lse
+        res += (mask, stat, full.astype(bool))
+    if want_row_stats:
+        res += (rstat,)
+    return res
 
 
 def dense(Q, K, V, causal=False, scale=None):

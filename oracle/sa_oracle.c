@@ -39,6 +39,10 @@
  *    scaled logit over the tile's visible pairs; only blocks whose every pair
  *    is visible ("full" blocks) may be skipped; a skipped block's keys leave
  *    G_i for every row i of the tile (so they leave the softmax denominator).
+ *    The episode's summary words the rule per query (each query's scores
+ *    decide which value blocks matter); that reading is built as an option:
+ *    a row also drops a full block when its own maximum over the block is
+ *    below the threshold, and the block is skipped when every row drops it.
  *
  * Steps follow the definitions in order: build G_i explicitly, compute logits
  * for j in G_i, max, exp, sum, normalise, weighted sum of V rows.  Two passes,
@@ -316,12 +320,24 @@ void ora_tile_blocks(const ora_pattern_t *p, int kind, int B, int H, int Hkv,
  * override: [B][H][T][n_kb] int8 (-1 = rule, 0 = keep, 1 = skip) or NULL.
  * keep_in_denominator: 1 = skipped keys' logits still enter the denominator
  *   (the variant reading; not the default).
+ * row_level: 1 = the per-query reading of the rule ("Block Sparse Flash
+ *   Attention", paper summary: the scores of each query decide which value
+ *   blocks matter): on top of the tile decisions, row i drops a full block of
+ *   its tile from G_i when its own maximum scaled logit over the block's keys
+ *   is below the threshold.  A tile's block is skipped (mask 2) exactly when
+ *   every row drops it, which is the tile rule's decision; partial blocks are
+ *   never dropped.  Not combined with keep_in_denominator.
+ * row_override: [n_rows][n_kb] int8 (-1 = rule, 0 = keep, 1 = drop) or NULL,
+ *   per requested row and key block (row_level only).
+ * row_stat_out: [n_rows][n_kb] (nullable, row_level only): the row's maximum
+ *   scaled logit over each full block of its tile, -inf for other blocks.
  * mask_out / stat_out / full_out: [B][H][T][n_kb] (nullable); only tiles
  *   that hold a requested row are written.  O: [n_rows][d], lse: [n_rows]. */
 void ora_prefill(const ora_pattern_t *p, int kind, int B, int H, int Hkv, int N,
                  int d, double scale, const void *Q, const void *K, const void *V,
                  const double *thresholds, const int8_t *override_mask,
-                 int keep_in_denominator, int64_t n_rows, const int32_t *rows,
+                 int keep_in_denominator, int row_level, const int8_t *row_override,
+                 double *row_stat_out, int64_t n_rows, const int32_t *rows,
                  double *O, double *lse, uint8_t *mask_out, double *stat_out,
                  uint8_t *full_out, int nthreads)
 {
@@ -380,6 +396,8 @@ void ora_prefill(const ora_pattern_t *p, int kind, int B, int H, int Hkv, int N,
         int32_t *G = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
         int32_t *Gk = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
         double *extra = (double *)malloc(sizeof(double) * (size_t)N);
+        double *rmax = (double *)malloc(sizeof(double) * (size_t)n_kb);
+        uint8_t *rdrop = (uint8_t *)malloc((size_t)n_kb);
         #pragma omp for schedule(dynamic, 16)
         for (int64_t r = 0; r < total; ++r) {
             int b, h, i;
@@ -390,10 +408,34 @@ void ora_prefill(const ora_pattern_t *p, int kind, int B, int H, int Hkv, int N,
             int nk = 0, ne = 0;
             int64_t q_off = (((int64_t)b * H + h) * N + i) * d;
             int64_t kv_off = ((int64_t)b * Hkv + hkv) * N * d;
-            const uint8_t *tm = need_tiles
-                ? tile_mask + (((int64_t)b * H + h) * T + i / p->block_q) * n_kb : NULL;
+            int64_t u_row = ((int64_t)b * H + h) * T + i / p->block_q;
+            const uint8_t *tm = need_tiles ? tile_mask + u_row * n_kb : NULL;
+            if (row_level && thresholds != NULL) {
+                /* the row's own maximum over each full block of its tile */
+                const int64_t *tc = tile_cnt + u_row * n_kb;
+                for (int kb = 0; kb < n_kb; ++kb) rmax[kb] = -INFINITY;
+                for (int k = 0; k < nG; ++k) {
+                    int j = G[k], kb = j / p->block_k;
+                    if (tc[kb] != (int64_t)p->block_q * p->block_k) continue;
+                    double acc = 0.0;
+                    for (int c = 0; c < d; ++c)
+                        acc += ld(Q, q_off + c, kind) * ld(K, kv_off + (int64_t)j * d + c, kind);
+                    if (scale * acc > rmax[kb]) rmax[kb] = scale * acc;
+                }
+                for (int kb = 0; kb < n_kb; ++kb) {
+                    int full = tc[kb] == (int64_t)p->block_q * p->block_k;
+                    int drop = full && rmax[kb] < thresholds[h];
+                    if (row_override != NULL && row_override[r * n_kb + kb] >= 0)
+                        drop = row_override[r * n_kb + kb] ? 1 : 0;
+                    rdrop[kb] = (uint8_t)drop;
+                    if (row_stat_out) row_stat_out[r * n_kb + kb] = full ? rmax[kb] : -INFINITY;
+                }
+            }
             for (int k = 0; k < nG; ++k) {
                 int j = G[k];
+                if (row_level && thresholds != NULL && tm && tm[j / p->block_k] != 2 &&
+                    rdrop[j / p->block_k])
+                    continue;   /* dropped by this row alone: the key leaves G_i */
                 if (tm && tm[j / p->block_k] == 2) {
                     if (keep_in_denominator) {
                         double acc = 0.0;
@@ -408,7 +450,7 @@ void ora_prefill(const ora_pattern_t *p, int kind, int B, int H, int Hkv, int N,
             row_attention(kind, Q, q_off, K, V, kv_off, d, scale, Gk, nk, extra, ne,
                           O + r * d, lse + r);
         }
-        free(G); free(Gk); free(extra);
+        free(G); free(Gk); free(extra); free(rmax); free(rdrop);
     }
     free(tile_needed); free(tile_mask); free(tile_stat); free(tile_cnt);
 }

@@ -475,3 +475,98 @@ def test_bsfa_skipped_keys_in_denominator_variant(oracle_mod):
     sb = sb.masked_fill(blk[:, None] != blk[None, :], float("-inf"))
     assert np.all(Ob == 0)
     assert np.max(np.abs(torch.logsumexp(sb, -1).numpy() - lb)) < 1e-10
+
+
+def _row_level_case(oracle_mod):
+    """Causal window of 300 over N=512: tiles hold full blocks and partial blocks
+    on both window edges."""
+    B, H, Hkv, N, d, Q, K, V = _bsfa_small(oracle_mod, seed=47)
+    p = oracle_mod.Pattern(causal=1, window=300, block_q=128, block_k=64)
+    return B, H, Hkv, N, d, Q, K, V, p
+
+
+def test_bsfa_row_level_extreme_thresholds(oracle_mod):
+    """Row-level reading: tau = -inf drops nothing (the static pattern, bit for
+    bit); tau = +inf drops every full block from every row, which is the tile
+    rule's result at +inf."""
+    B, H, Hkv, N, d, Q, K, V, p = _row_level_case(oracle_mod)
+    O0, l0 = oracle_mod.prefill(p, Q, K, V)
+    O1, l1 = oracle_mod.prefill(p, Q, K, V, thresholds=np.full(H, -np.inf), row_level=True)
+    assert np.array_equal(O0, O1) and np.array_equal(l0, l1)
+    O2, l2 = oracle_mod.prefill(p, Q, K, V, thresholds=np.full(H, np.inf), row_level=True)
+    O3, l3 = oracle_mod.prefill(p, Q, K, V, thresholds=np.full(H, np.inf))
+    assert np.array_equal(O2, O3) and np.array_equal(l2, l3)
+
+
+def _median_tau(stat, full, H):
+    """A threshold per head between two consecutive full-block statistics near
+    their median (far from every statistic, so rounding cannot move a decision)."""
+    tau = np.empty(H)
+    for h in range(H):
+        v = np.sort(stat[:, h][full[:, h]])
+        k = (len(v) - 1) // 2
+        tau[h] = 0.5 * (v[k] + v[k + 1])
+    return tau
+
+
+def test_bsfa_row_level_against_numpy_brute_force(oracle_mod):
+    """Row-level reading against a numpy restatement of its definition: scores
+    by einsum, G_i by the Python predicate, tile fullness by counting visible
+    pairs, each row's maximum over each full block, the dropped blocks' keys
+    removed from G_i, softmax over what is left.  Also: the skip set (blocks
+    every row drops) is the tile rule's, and a row's per-block maxima reduce to
+    the tile statistic."""
+    B, H, Hkv, N, d, Q, K, V, p = _row_level_case(oracle_mod)
+    scale = 1 / math.sqrt(d)
+    _, _, mask_t, stat_t, full_t = oracle_mod.prefill(p, Q, K, V, want_blocks=True,
+                                                      thresholds=np.full(H, -np.inf))
+    tau = _median_tau(stat_t, full_t, H)
+    O, lse, mask_r, stat_r, full_r, rstat = oracle_mod.prefill(
+        p, Q, K, V, thresholds=tau, row_level=True, want_blocks=True, want_row_stats=True)
+    _, _, mask_tile, _, _ = oracle_mod.prefill(p, Q, K, V, thresholds=tau, want_blocks=True)
+    assert np.array_equal(mask_r, mask_tile)
+    vis = np.array([[oracle_mod.visible_py(p, N, 0, i, j) for j in range(N)] for i in range(N)])
+    T, n_kb = N // 128, N // 64
+    full = np.array([[vis[t * 128:(t + 1) * 128, kb * 64:(kb + 1) * 64].all()
+                      for kb in range(n_kb)] for t in range(T)])
+    assert np.array_equal(full_r[0, 0], full)
+    dropped_any = 0
+    for h in range(H):
+        S = scale * np.einsum("id,jd->ij", Q[0, h], K[0, 0])
+        for i in range(N):
+            t = i // 128
+            keep = vis[i].copy()
+            for kb in range(n_kb):
+                if not full[t, kb]:
+                    assert rstat.reshape(H, N, n_kb)[h, i, kb] == -np.inf
+                    continue
+                rm = S[i, kb * 64:(kb + 1) * 64].max()
+                assert rstat.reshape(H, N, n_kb)[h, i, kb] == pytest.approx(rm, abs=1e-12)
+                if rm < tau[h]:
+                    keep[kb * 64:(kb + 1) * 64] = False
+                    dropped_any += mask_r[0, h, t, kb] == 1
+            s = S[i, keep]
+            w = np.exp(s - s.max())
+            out = (w / w.sum()) @ V[0, 0][keep]
+            assert np.max(np.abs(out - O[0, h, i])) < 1e-12
+            assert abs(lse[0, h, i] - (s.max() + np.log(w.sum()))) < 1e-12
+        # the tile statistic is the largest of its rows' maxima
+        rs = rstat.reshape(H, N, n_kb)[h].reshape(T, 128, n_kb).max(axis=1)
+        assert np.allclose(rs[full], stat_t[0, h][full], rtol=0, atol=1e-12)
+    # the reading changes something: rows drop blocks the tile keeps
+    assert dropped_any > 0
+
+
+def test_bsfa_row_level_override_keep_is_the_tile_rule(oracle_mod):
+    """Forcing every row to keep (row override 0) leaves the tile rule's result."""
+    B, H, Hkv, N, d, Q, K, V, p = _row_level_case(oracle_mod)
+    _, _, _, stat_t, full_t = oracle_mod.prefill(p, Q, K, V, want_blocks=True,
+                                                 thresholds=np.full(H, -np.inf))
+    tau = _median_tau(stat_t, full_t, H)
+    n_kb = N // 64
+    keep_all = np.zeros((B * H * N, n_kb), np.int8)
+    O1, l1 = oracle_mod.prefill(p, Q, K, V, thresholds=tau, row_level=True, row_override=keep_all)
+    O2, l2 = oracle_mod.prefill(p, Q, K, V, thresholds=tau)
+    assert np.array_equal(O1, O2) and np.array_equal(l1, l2)
+    O3, l3 = oracle_mod.prefill(p, Q, K, V, thresholds=tau, row_level=True)
+    assert not np.array_equal(O3, O2)
