@@ -2,6 +2,14 @@
 """Benchmark of the block-sparse attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--no-secondary]
+
+The headline workload (the default) is bsfa_causal: causal prefill at N=32768
+with the Block-Sparse-FlashAttention rule.  The same run then times every other
+workload of the metric (mistral_swa, longformer_bigbird, gather_decode,
+tiny_static) and the extensions (bsfa_denominator, dilated_swa, window_decode,
+topk_decode), each with its own roofline, clocks and traffic, under
+secondary.workloads of the JSON line (--no-secondary skips them).
 
 One step = one pass of the hot path over one batch of synthetic input: for a
 prefill workload one sparse_attn_prefill_plan launch (pattern compile and, for
@@ -21,7 +29,9 @@ The printed JSON line carries the headline metric, an end-to-end number
 through the same C-ABI call with host (pinned) buffers and the host<->device
 copies inside the timed region, the roofline of the dominant kernel against
 the measured peaks, SM clocks sampled during the timed region and the CPU
-baseline (the fp64 oracle on a bounded sample, rank 0, N=1 only).
+baseline (the fp64 oracle on a bounded sample, rank 0, N=1 only; for the
+block-skip workloads the oracle uses thresholds it calibrates itself on a
+sample of the calibration draw).
 
 --impl reference times the fp64 CPU oracle as it stands on the host cores, on
 the same workload and metric (bounded samples per step), and prints the same
@@ -45,6 +55,7 @@ sys.path.insert(0, ROOT)
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+NEAR_BAND = 1e-3   # block statistics this close to the threshold may be decided either way
 
 
 # ------------------------------------------------------------------ helpers --
@@ -187,9 +198,23 @@ def setup_prefill(w, device, torch, sa, workloads):
         thresholds = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
         del Qc, Kc
         mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=device)
-        plan.prefill(Q, K, V, thresholds=thresholds, block_mask=mask)
+        stat = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.float32, device=device)
+        plan.prefill(Q, K, V, thresholds=thresholds, block_mask=mask, block_stat=stat)
         sa.check_device_error()
         skipped = int((mask == 2).sum())
+        # blocks whose statistic lies within NEAR_BAND of their head's threshold: the
+        # ones a CPU recomputation in another precision may decide the other way
+        # (the parity tests compare whole heads with the oracle outside this band)
+        row_ptr, kb, fl, _, H_pat, T = sa.compile_pattern(pat, w.H, w.N)
+        full = torch.zeros((H_pat, T, plan.n_kb), dtype=torch.bool)
+        for hp in range(H_pat):
+            for t in range(T):
+                a, e = row_ptr[hp * T + t], row_ptr[hp * T + t + 1]
+                full[hp, t, torch.from_numpy(kb[a:e][fl[a:e]]).long()] = True
+        full = full.to(device).unsqueeze(0).expand(w.B, w.H if H_pat == 1 else -1, -1, -1)
+        near = (stat - thresholds.view(1, -1, 1, 1)).abs() <= NEAR_BAND
+        extra["near_threshold_blocks"] = int((near & full).sum())
+        del stat, near, full
         kept_desc = plan.info["blocks_desc"] - skipped
         skipped_pairs = skipped * w.block_q * w.block_k
         extra["blocks_skipped"] = skipped
@@ -334,9 +359,11 @@ def setup_topk_decode(w, device, torch, sa, workloads):
 
 
 # ------------------------------------------------------------- CPU baseline --
-def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
+def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None, thresholds=None,
+                    threshold_note=""):
     """Times the fp64 oracle as it stands on the host cores over a bounded sample
-    of the workload; returns (value in the workload's unit, cores, description)."""
+    of the workload; returns (value in the workload's unit, cores, description).
+    thresholds: the block-skip workloads' per-head thresholds (oracle_thresholds)."""
     import numpy as np
     import torch
     import oracle
@@ -415,51 +442,182 @@ def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None):
             n = min(4096, n * 2)
         gbs = done_rows * (2 * w.d * 2 + 4) / t_total / 1e9
         return gbs, cores, f"{done_rows // w.n_idx} (sequence, head) sets, {done_rows} rows"
-    # prefill: whole 128-row tiles, so computed-block FLOPs are exact for the sample
+    # prefill: whole query tiles of the descriptor's height (block_q rows of one
+    # residue class for a dilated window).  The computed-block FLOPs of the
+    # sample are counted from the oracle's own enumeration of G_i (build_G) at
+    # the descriptor's block granularity, and for the block-skip rule from the
+    # oracle's own block decisions; nothing here touches the CUDA library.
     Q, K, V, tab = (device_tensors if device_tensors is not None
                     else workloads.prefill_inputs(w, device="cpu"))
-    if isinstance(Q, torch.Tensor):
-        Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
+    Qh, Kh, Vh = (Q.cpu(), K.cpu(), V.cpu()) if isinstance(Q, torch.Tensor) else (Q, K, V)
     opat = oracle.Pattern(**w.pattern_fields(), random_table=tab)
-    thresholds = None
-    if w.bsfa:
-        thresholds = np.zeros(w.H)   # the rule's statistic pass is what is timed
-    from block_sparse_attention_29_b200 import compile_pattern, Pattern
-    row_ptr, kb, full, cnt, H_pat, T = compile_pattern(Pattern(**w.pattern_fields(),
-                                                               random_table=tab), w.H, w.N)
-    # a dilated window's tiles are 128 positions of one residue class r:
-    # rows (t*128 + m)*k + r
+    if w.bsfa and thresholds is None:
+        raise RuntimeError("the block-skip workloads need the oracle's thresholds")
     k = max(1, w.dilation)
     n_pos = w.N // k
-    flops_done, t_total, tiles_done, n = 0, 0.0, 0, 1
+    bq, bk = w.block_q, w.block_k
+    T = -(-n_pos // bq)
+    flops_done, t_total, tiles_done, n, blocks_done = 0, 0.0, 0, 1, 0
+    listed_of = {}   # (head or 0, tile, residue class) -> listed blocks (the lists repeat)
+
+    def listed_blocks(h, t, r):
+        key = (h if w.n_random > 0 else 0, t, r)
+        if key not in listed_of:
+            kbs = set()
+            for mm in range(t * bq, min(n_pos, t * bq + bq)):
+                G = oracle.build_G(opat, w.N, h, mm * k + r)
+                kbs.update(np.unique((G // k) // bk).tolist())
+            listed_of[key] = len(kbs)
+        return listed_of[key]
     while t_total < seconds:
         tiles = [(int(g.integers(w.B)), int(g.integers(w.H)), int(g.integers(T)),
                   int(g.integers(k))) for _ in range(n)]
         rows = np.array([(b, h, m * k + r) for b, h, t, r in tiles
-                         for m in range(t * 128, min(n_pos, t * 128 + 128))], np.int32)
+                         for m in range(t * bq, min(n_pos, t * bq + bq))], np.int32)
         t0 = time.perf_counter()
-        oracle.prefill(opat, Qh, Kh, Vh, thresholds=thresholds, rows=rows, nthreads=cores,
-                       keep_in_denominator=bool(w.skipped_in_denominator))
+        res = oracle.prefill(opat, Qh, Kh, Vh, thresholds=thresholds, rows=rows, nthreads=cores,
+                             keep_in_denominator=bool(w.skipped_in_denominator),
+                             want_blocks=bool(w.bsfa))
         t_total += time.perf_counter() - t0
-        for b, h, t, _r in tiles:
-            hp = h if H_pat > 1 else 0
-            nb = int(row_ptr[hp * T + t + 1] - row_ptr[hp * T + t])
-            flops_done += 4 * 128 * 64 * w.d * nb
+        for b, h, t, r in tiles:
+            if w.bsfa:
+                m = res[2][b, h, t]
+                listed, kept = int((m != 0).sum()), int((m == 1).sum())
+            else:
+                listed = kept = listed_blocks(h, t, r)
+            flops_done += 2 * bq * bk * w.d * (listed + kept)
+            blocks_done += listed
         tiles_done += n
         n = min(64, n * 2)
-    return flops_done / t_total / 1e12, cores, f"{tiles_done} whole 128-row query tiles"
+    what = f"{tiles_done} whole {bq}-row query tiles ({blocks_done} listed {bq}x{bk} blocks)"
+    if w.bsfa:
+        what += ", thresholds " + threshold_note
+    return flops_done / t_total / 1e12, cores, what
+
+
+def oracle_thresholds(w, tiles_per_head=4, nthreads=0):
+    """Per-head thresholds of the block-skip rule computed by the oracle alone:
+    the lower median of the full-block statistics of a seeded sample of the
+    calibration draw's query tiles (tiles_per_head per head, spread over the
+    sequence).  Used by the oracle's timing legs, which cannot afford the
+    statistics of the whole calibration draw."""
+    import numpy as np
+    import oracle
+    from block_sparse_attention_29_b200 import workloads
+    Qc, Kc, _, tab = workloads.calibration_inputs(w, device="cpu")
+    opat = oracle.Pattern(**w.pattern_fields(), random_table=tab)
+    T = -(-w.N // w.block_q)
+    g = np.random.default_rng(77)
+    tiles = [(b, h, int(t)) for b in range(w.B) for h in range(w.H)
+             for t in g.choice(np.arange(T // 4, T), size=tiles_per_head, replace=False)]
+    full, stat, _ = oracle.block_stats(opat, Qc, Kc, tiles=np.array(tiles, np.int32),
+                                       nthreads=nthreads)
+    return (oracle.calibrate_thresholds(full, stat),
+            f"from the oracle's statistics of {tiles_per_head} calibration tiles per head")
 
 
 # --------------------------------------------------------------------- main --
+HEADLINE = "bsfa_causal"
+# Timed after the headline in the same run: the other four configurations of
+# the metric (tiny static pattern, Mistral window, Longformer/BigBird, index-set
+# gather), then the extensions (the block-skip variant, dilated window, window
+# decode, top-K decode).
+SECONDARY = ("mistral_swa", "longformer_bigbird", "gather_decode", "tiny_static",
+             "bsfa_denominator", "dilated_swa", "window_decode", "topk_decode")
+SECONDARY_MIN_S = 0.3   # each secondary workload's timed region lasts at least this long
+
+
+def setup_for(w, workloads):
+    if isinstance(w, workloads.WindowDecodeWorkload):
+        return setup_window_decode
+    if isinstance(w, workloads.TopkDecodeWorkload):
+        return setup_topk_decode
+    if isinstance(w, workloads.GatherWorkload):
+        return setup_gather
+    return setup_prefill
+
+
+def time_steps(S, steps, warmup, stream, flush, torch, sa, dist, device, clock_index):
+    """W untimed warm-up steps, then exactly `steps` steps between a barrier and
+    a synchronize on both sides; each step's launches are timed with CUDA events
+    on their stream, L2 flushed before every step (outside the events).
+    Returns (per-step ms, total ms max over ranks, clock summary)."""
+    for _ in range(warmup):
+        flush.zero_()
+        S["step"](stream)
+    sa.check_device_error()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(clock_index) as clk:
+        for k in range(steps):
+            flush.zero_()
+            starts[k].record(stream)
+            S["step"](stream)
+            ends[k].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    sa.check_device_error()
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(per_step), dist, device)
+    return per_step, total_ms, clk.summary()
+
+
+def summarize(S, w, world, steps, warmup, per_step, total_ms, clocks, peaks, peak_src):
+    """Metric value, roofline of the dominant kernel and the secondary figures."""
+    ms_per_step = total_ms / steps
+    per_launch_s = ms_per_step / 1e3
+    if S["unit"] == "TFLOP/s":
+        value = aggregate_rate(world, S["flops"], per_launch_s, 1e12)
+        achieved = S["flops"] / per_launch_s / 1e12
+        peak = peaks["bf16_tflops"]
+        roof_unit = "TFLOP/s"
+    else:
+        value = aggregate_rate(world, S["algo_bytes"], per_launch_s, 1e9)
+        achieved = value / world
+        peak = peaks["hbm_gbs"]
+        roof_unit = "GB/s"
+    sha = kernel_source_sha(S["kernel_files"])
+    out = {
+        "metric": S["metric"], "value": round(value, 3), "unit": S["unit"], "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": round(ms_per_step, 5),
+        "roofline": {"bound": S["bound"], "achieved": round(achieved, 3), "peak": peak,
+                     "unit": roof_unit, "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if roof_unit == 'TFLOP/s' else 'hbm_gbs'})",
+                     "traffic": recorded_traffic(S["kernel"], w.name, sha),
+                     "kernel": S["kernel"], "kernel_source_sha": sha},
+        "clocks": clocks,
+        "per_step_ms": {"min": round(min(per_step), 5), "median": round(statistics.median(per_step), 5),
+                        "max": round(max(per_step), 5)},
+    }
+    if S["unit"] == "TFLOP/s":
+        out["secondary"] = {
+            "dense_equiv_tflops": round(world * S["dense_flops"] / per_launch_s / 1e12, 3),
+            "exact_pair_tflops": round(world * S["exact_flops"] / per_launch_s / 1e12, 3),
+            "pct_bf16_peak_burst": round(100 * achieved / peaks["bf16_tflops"], 2),
+            "pct_bf16_peak_sustained": round(100 * achieved / peaks.get("bf16_tflops_sustained", 1400.0), 2),
+            "computed_block_flops": S["flops"], **S["extra"]}
+    else:
+        out["secondary"] = {"pct_hbm_peak": round(100 * achieved / peaks["hbm_gbs"], 2),
+                            "algorithmic_bytes": S["algo_bytes"], **S["extra"]}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mistral_swa")
+    ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="time the chosen workload only (the secondary workloads are timed "
+                         "after the headline by default)")
     ap.add_argument("--sequences", type=int, default=0,
                     help="decode workloads: run this many sequences instead of the workload's "
                          "(a reduced case of the same kernels, e.g. for counter captures)")
@@ -493,40 +651,13 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
 
-    if isinstance(w, workloads.WindowDecodeWorkload):
-        setup = setup_window_decode
-    elif isinstance(w, workloads.TopkDecodeWorkload):
-        setup = setup_topk_decode
-    else:
-        setup = setup_gather if isinstance(w, workloads.GatherWorkload) else setup_prefill
-    S = setup(w, device, torch, sa, workloads)
+    S = setup_for(w, workloads)(w, device, torch, sa, workloads)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        S["step"](stream)
-    sa.check_device_error()
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        for k in range(args.steps):
-            flush.zero_()
-            starts[k].record(stream)
-            S["step"](stream)
-            ends[k].record(stream)
-        torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    sa.check_device_error()
-    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(per_step)
-    total_ms = max_over_ranks(total_ms, dist, device)
-    ms_per_step = total_ms / args.steps
+    per_step, total_ms, clocks = time_steps(S, args.steps, args.warmup, stream, flush, torch, sa,
+                                            dist, device, local_rank)
 
     # end to end: the same call with host buffers, copies inside the timed region
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -543,26 +674,15 @@ def main():
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device) / args.steps
     sa.check_device_error()
 
-    peaks, peak_src = load_peaks()
-    per_launch_s = ms_per_step / 1e3
+    head = summarize(S, w, world, args.steps, args.warmup, per_step, total_ms, clocks, peaks,
+                     peak_src)
     if S["unit"] == "TFLOP/s":
-        value = aggregate_rate(world, S["flops"], per_launch_s, 1e12)
         e2e_value = aggregate_rate(world, S["flops"], e2e_ms / 1e3, 1e12)
-        achieved = S["flops"] / per_launch_s / 1e12
-        peak = peaks["bf16_tflops"]
-        roof_unit = "TFLOP/s"
     else:
-        value = aggregate_rate(world, S["algo_bytes"], per_launch_s, 1e9)
         e2e_value = aggregate_rate(world, S["algo_bytes"], e2e_ms / 1e3, 1e9)
-        achieved = value / world
-        peak = peaks["hbm_gbs"]
-        roof_unit = "GB/s"
-    sha = kernel_source_sha(S["kernel_files"])
-    traffic = recorded_traffic(S["kernel"], w.name, sha)
-
     out = {
-        "metric": S["metric"], "value": round(value, 3), "unit": S["unit"], "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "metric": head["metric"], "value": head["value"], "unit": head["unit"], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, device-generated; see block_sparse_attention_29_b200/workloads.py)",
         "config": config_of(w, world),
@@ -570,24 +690,9 @@ def main():
                 "h2d_bytes_per_step": S["h2d"], "d2h_bytes_per_step": S["d2h"],
                 "ms_per_step": round(e2e_ms, 5)},
         "gpu_launches": args.steps * S.get("launches_per_step", 1),
-        "roofline": {"bound": S["bound"], "achieved": round(achieved, 3), "peak": peak,
-                     "unit": roof_unit, "frac": round(achieved / peak, 4),
-                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if roof_unit == 'TFLOP/s' else 'hbm_gbs'})",
-                     "traffic": traffic, "kernel": S["kernel"], "kernel_source_sha": sha},
-        "clocks": clk.summary(),
-        "per_step_ms": {"min": round(min(per_step), 5), "median": round(statistics.median(per_step), 5),
-                        "max": round(max(per_step), 5)},
+        "roofline": head["roofline"], "clocks": head["clocks"], "per_step_ms": head["per_step_ms"],
+        "secondary": head["secondary"],
     }
-    if S["unit"] == "TFLOP/s":
-        out["secondary"] = {
-            "dense_equiv_tflops": round(world * S["dense_flops"] / per_launch_s / 1e12, 3),
-            "exact_pair_tflops": round(world * S["exact_flops"] / per_launch_s / 1e12, 3),
-            "pct_bf16_peak_burst": round(100 * achieved / peaks["bf16_tflops"], 2),
-            "pct_bf16_peak_sustained": round(100 * achieved / peaks.get("bf16_tflops_sustained", 1400.0), 2),
-            "computed_block_flops": S["flops"], **S["extra"]}
-    else:
-        out["secondary"] = {"pct_hbm_peak": round(100 * achieved / peaks["hbm_gbs"], 2),
-                            "algorithmic_bytes": S["algo_bytes"], **S["extra"]}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         if isinstance(w, (workloads.GatherWorkload, workloads.WindowDecodeWorkload,
@@ -597,9 +702,39 @@ def main():
         else:
             Q, K, V, _ = S["tensors"]
             dt = (Q, K, V, S["tab"])
-        val, cores, sample = cpu_oracle_rate(w, args.cpu_seconds, device_tensors=dt)
+        th, note = (oracle_thresholds(w) if getattr(w, "bsfa", False) else (None, ""))
+        val, cores, sample = cpu_oracle_rate(w, args.cpu_seconds, device_tensors=dt,
+                                             thresholds=th, threshold_note=note)
         out["cpu_baseline"] = {"value": round(val, 6), "unit": S["unit"], "cores": cores,
                                "kind": "oracle", "sample": sample}
+    S = None
+    torch.cuda.empty_cache()
+
+    if args.workload == HEADLINE and not args.no_secondary:
+        table = {}
+        for name in SECONDARY:
+            ws = workloads.WORKLOADS[name]
+            Ss = setup_for(ws, workloads)(ws, device, torch, sa, workloads)
+            # steps: enough for SECONDARY_MIN_S of timed work (clock samples), at least --steps
+            probe, _, _ = time_steps(Ss, 3, args.warmup, stream, flush, torch, sa, dist, device,
+                                     local_rank)
+            est = max(1e-3, statistics.median(probe))
+            steps = min(2000, max(args.steps, math.ceil(1e3 * SECONDARY_MIN_S / est)))
+            steps = int(max_over_ranks(steps, dist, device))
+            ps, tot, clk = time_steps(Ss, steps, 3, stream, flush, torch, sa, dist, device,
+                                      local_rank)
+            r = summarize(Ss, ws, world, steps, 3, ps, tot, clk, peaks, peak_src)
+            r["config"] = config_of(ws, world)
+            r["gpu_launches"] = steps * Ss.get("launches_per_step", 1)
+            table[name] = r
+            Ss = None
+            torch.cuda.empty_cache()
+        out["secondary"]["workloads"] = table
+        out["secondary"]["workloads_note"] = (
+            "each timed like the headline (CUDA events per step, L2 flushed before every step, "
+            "clocks sampled during its own timed region); end-to-end and CPU baseline are "
+            "measured for the headline only")
+
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist:
@@ -657,14 +792,17 @@ def run_reference(args, w, world):
         w = ws
     else:
         dt = workloads.prefill_inputs(w, device="cpu")
+    # the block-skip rule's thresholds, calibrated by the oracle itself (untimed)
+    th, note = (oracle_thresholds(w) if getattr(w, "bsfa", False) else (None, ""))
     budget = 60.0
     per_step = max(1.0, budget / (args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_oracle_rate(w, per_step / 4, device_tensors=dt)
+        cpu_oracle_rate(w, per_step / 4, device_tensors=dt, thresholds=th, threshold_note=note)
     vals, cores, sample = [], None, None
     t0 = time.perf_counter()
     for k in range(args.steps):
-        v, cores, sample = cpu_oracle_rate(w, per_step, sample_seed=k + 1, device_tensors=dt)
+        v, cores, sample = cpu_oracle_rate(w, per_step, sample_seed=k + 1, device_tensors=dt,
+                                           thresholds=th, threshold_note=note)
         vals.append(v)
     elapsed = time.perf_counter() - t0
     value = statistics.mean(vals)
