@@ -112,6 +112,29 @@ int make_tmap(CUtensorMap* m, const void* base, int d, int N, int BH, int rows, 
   return SA_OK;
 }
 
+// Shape and descriptor checks shared by every prefill entry point.
+int check_shapes(const sa_pattern_t* pat, int B, int H, int Hkv, int N, int d) {
+  if (!pat) return set_error(SA_ERR_INVALID_ARG, "pattern descriptor is NULL");
+  if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0)
+    return set_error(SA_ERR_INVALID_ARG, "B, H, H_kv and N must be positive");
+  if (H % Hkv != 0) return set_error(SA_ERR_INVALID_ARG, "H = %d is not a multiple of H_kv = %d", H, Hkv);
+  if (d != 64 && d != 128) return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
+  if (pat->block_k != kTileK)
+    return set_error(SA_ERR_UNSUPPORTED, "block_k = %d (the kernels use 64-key blocks)", pat->block_k);
+  if (pat->block_q != 64 && pat->block_q != 128)
+    return set_error(SA_ERR_UNSUPPORTED, "block_q = %d (64 or 128 supported)", pat->block_q);
+  if (pat->n_random > 0 && pat->random_table && (pat->random_block <= 0 || pat->random_block % kTileK))
+    return set_error(SA_ERR_UNSUPPORTED, "random_block = %d must be a positive multiple of 64",
+                     pat->random_block);
+  if (N >= (1 << 28)) return set_error(SA_ERR_UNSUPPORTED, "N = %d too large", N);
+  const int dil = pat->dilation > 1 ? pat->dilation : 1;
+  const int64_t units = int64_t(B) * dil * H * ((N / dil + kTileQ - 1) / kTileQ);
+  if (units > INT32_MAX) return set_error(SA_ERR_UNSUPPORTED, "B*H*tiles too large");
+  if (int64_t(B) * H > 65535 || int64_t(B) * Hkv > 65535)
+    return set_error(SA_ERR_UNSUPPORTED, "B*H must not exceed 65535");
+  return SA_OK;
+}
+
 }  // namespace sa
 
 // ================================================================= plans ==
@@ -159,28 +182,6 @@ int upload(T** dst, const T* src, size_t n) {
     e = cudaMemcpy(*dst, src, n * sizeof(T), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) return cuda_error(e, "cudaMemcpy");
   }
-  return SA_OK;
-}
-
-int check_shapes(const sa_pattern_t* pat, int B, int H, int Hkv, int N, int d) {
-  if (!pat) return set_error(SA_ERR_INVALID_ARG, "pattern descriptor is NULL");
-  if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0)
-    return set_error(SA_ERR_INVALID_ARG, "B, H, H_kv and N must be positive");
-  if (H % Hkv != 0) return set_error(SA_ERR_INVALID_ARG, "H = %d is not a multiple of H_kv = %d", H, Hkv);
-  if (d != 64 && d != 128) return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
-  if (pat->block_k != kTileK)
-    return set_error(SA_ERR_UNSUPPORTED, "block_k = %d (the kernels use 64-key blocks)", pat->block_k);
-  if (pat->block_q != 64 && pat->block_q != 128)
-    return set_error(SA_ERR_UNSUPPORTED, "block_q = %d (64 or 128 supported)", pat->block_q);
-  if (pat->n_random > 0 && pat->random_table && (pat->random_block <= 0 || pat->random_block % kTileK))
-    return set_error(SA_ERR_UNSUPPORTED, "random_block = %d must be a positive multiple of 64",
-                     pat->random_block);
-  if (N >= (1 << 28)) return set_error(SA_ERR_UNSUPPORTED, "N = %d too large", N);
-  const int dil = pat->dilation > 1 ? pat->dilation : 1;
-  const int64_t units = int64_t(B) * dil * H * ((N / dil + kTileQ - 1) / kTileQ);
-  if (units > INT32_MAX) return set_error(SA_ERR_UNSUPPORTED, "B*H*tiles too large");
-  if (int64_t(B) * H > 65535 || int64_t(B) * Hkv > 65535)
-    return set_error(SA_ERR_UNSUPPORTED, "B*H must not exceed 65535");
   return SA_OK;
 }
 

@@ -145,6 +145,9 @@ int compile_pattern(const sa_pattern_t* pat, int H, int N, int tile_q, int tile_
                     CompiledPattern* out);
 // Validates the descriptor fields that do not depend on the kernel.
 int validate_pattern(const sa_pattern_t* pat, int H, int N);
+// Shapes and the descriptor fields the kernels constrain (head dim, block
+// sizes, random-block granularity, grid and index limits); SA_OK or an error.
+int check_shapes(const sa_pattern_t* pat, int B, int H, int Hkv, int N, int d);
 // Work order of the B*H*T units (unit = (b*H + h)*T + t): units longer than
 // half a CTA's share first (longest first), the rest tile-major or
 // K/V-group-major (see kv_bytes), the query heads of a group adjacent.

@@ -8,14 +8,20 @@
 // whole device, or a runtime that forbids allocation on its inference path.
 // This entry point compiles the pattern on the host and copies the result into
 // a fixed, file-scope device array instead, then launches the same prefill
-// kernel.  The array is static device memory of kNoAllocScratchBytes, created
-// when the library is loaded and held on every device until the process
-// exits.
+// kernel.  The array is static device memory of kNoAllocScratchBytes.  CUDA
+// loads the library's device code lazily, so the array is reserved on a device
+// when the library's code is first used there (for a caller that only uses
+// this entry point: its first call) and held until the process exits.  A
+// caller whose device memory is about to be handed to an external pool should
+// make one call (a warm-up) before the pool takes the device.
 //
 // Set-up: the first call on a device, with that device current, looks up the
 // array's device address with cudaGetSymbolAddress (the array's name in host
 // code is only a host-side stand-in, not a device address).  Make that first
 // call before any stream capture begins.
+//
+// Every argument and size check, the size limit included, runs on the host
+// before the first CUDA call, so a rejected call queues no device work.
 //
 // Sharing: every call uses the same array and leaves the last call's contents
 // in it.  The plan data is rewritten in full by each call; the two work-queue
@@ -74,22 +80,15 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   if ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) |
        reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(O)) & 15u)
     return set_error(SA_ERR_INVALID_ARG, "Q, K, V and O must be 16-byte aligned");
-  if (B <= 0 || H <= 0 || H_kv <= 0 || N <= 0)
-    return set_error(SA_ERR_INVALID_ARG, "B, H, H_kv and N must be positive");
-  if (H % H_kv != 0) return set_error(SA_ERR_INVALID_ARG, "H = %d is not a multiple of H_kv = %d", H, H_kv);
-  if (d != 64 && d != 128) return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
-  if (pat->block_k != kTileK || (pat->block_q != 64 && pat->block_q != 128))
-    return set_error(SA_ERR_UNSUPPORTED, "block_q must be 64 or 128 and block_k 64");
+  int rc = check_shapes(pat, B, H, H_kv, N, d);
+  if (rc) return rc;
   if (pat->thresholds && pat->block_q != kTileQ)
     return set_error(SA_ERR_UNSUPPORTED, "the block-skip rule needs block_q = 128");
   const bool rnd = pat->n_random > 0 && pat->random_table != nullptr;
-  if (rnd && (pat->random_block <= 0 || pat->random_block % kTileK))
-    return set_error(SA_ERR_UNSUPPORTED, "random_block must be a positive multiple of 64");
-  if (int64_t(B) * H > 65535) return set_error(SA_ERR_UNSUPPORTED, "B*H must not exceed 65535");
 
   // Host compile (host memory only).
   CompiledPattern cp;
-  int rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
+  rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
   if (rc) return rc;
   const int T = cp.T;
   const bool pair = false;   // the single-head kernel (the default of the plan API)

@@ -296,10 +296,14 @@ int64_t sparse_attn_window_slot(int64_t j, int window, int n_global);
  * an external pool or allocator, or runtimes that forbid allocation on the
  * inference path.  Same arguments and result as sparse_attn_prefill (block
  * mask output excepted); the compiled pattern is not cached but rebuilt on the
- * host each call and copied into a fixed 8 MiB static device array that the
- * library holds on every device until the process exits.  Patterns whose
- * block lists, work order and random table need more than 8 MiB are rejected
- * with SA_ERR_INVALID_ARG.  The first call on a device looks up the array's
+ * host each call and copied into a fixed 8 MiB static device array.  CUDA
+ * loads the library's device code lazily, so the array is reserved on a
+ * device when that code is first used there (for a caller of this entry point
+ * alone: its first call) and held until the process exits; make a warm-up call
+ * before an external pool takes the rest of the device.  Patterns whose block
+ * lists, work order and random table need more than 8 MiB are rejected with
+ * SA_ERR_INVALID_ARG; every check runs on the host before the first CUDA call,
+ * so a rejected call queues no device work.  The first call on a device looks up the array's
  * device address (with that device current); make it before any stream
  * capture.  Every call reuses the array: calls that can overlap on the GPU
  * (different streams without ordering) race; calls on one stream do not.

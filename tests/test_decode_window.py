@@ -112,3 +112,38 @@ def test_decode_window_rejects_other_patterns(product):
                                           torch.zeros((1, 1, 9, 64), dtype=torch.bfloat16),
                                           torch.zeros((1, 1, 9, 64), dtype=torch.bfloat16),
                                           torch.zeros((1,), dtype=torch.int32), pat)
+
+
+@pytest.mark.gpu
+@pytest.mark.slow
+def test_decode_window_full_size(product, oracle_mod, cuda):
+    """window_decode at its full size (64 sequences, H=32, H_kv=8, d=128, W=4096,
+    4 globals, positions up to 131071): every (sequence, head) output and lse
+    against the oracle's gather over G_p, with G_p enumerated by the oracle from
+    the pattern and its keys read from their cache slots (the layout: key j in
+    slot j for j < g, else g + j mod W)."""
+    from block_sparse_attention_29_b200.workloads import WORKLOADS, window_decode_inputs
+    w = WORKLOADS["window_decode"]
+    Q, Kc, Vc, pos = window_decode_inputs(w, device=cuda)
+    pat = product.Pattern(causal=1, window=w.window, n_global=w.n_global)
+    lse = torch.empty((w.S, w.H), dtype=torch.float32, device=cuda)
+    O = product.sparse_attn_decode_window(Q, Kc, Vc, pos, pat, lse=lse)
+    product.check_device_error()
+
+    opat = oracle_mod.Pattern(causal=1, window=w.window, n_global=w.n_global)
+    positions = pos.cpu().numpy()
+    assert positions.max() <= w.max_pos and positions.min() >= w.window + w.n_global
+    n = w.window + w.n_global
+    Kk = torch.empty((w.S, w.H_kv, n, w.d), dtype=torch.bfloat16)
+    Vk = torch.empty_like(Kk)
+    for s, p in enumerate(positions):
+        G = oracle_mod.build_G(opat, int(p) + 1, 0, int(p))
+        assert len(G) == n and G[0] == 0 and G[-1] == p
+        slots = np.where(G < w.n_global, G, w.n_global + G % w.window)
+        ix = torch.from_numpy(slots.astype(np.int64)).to(cuda)
+        Kk[s] = Kc[s][:, ix].cpu()
+        Vk[s] = Vc[s][:, ix].cpu()
+    idx = np.broadcast_to(np.arange(n, dtype=np.int32), (w.S, w.H, n)).copy()
+    Or, lr = oracle_mod.gather(Q.cpu(), Kk, Vk, idx)
+    assert_close(O, Or)
+    assert_close(lse, lr, what="lse")
