@@ -186,17 +186,21 @@ def prefill_accounting(w, info, kept_desc=None, skipped_pairs=0):
 def setup_prefill(w, device, torch, sa, workloads):
     Q, K, V, tab = workloads.prefill_inputs(w, device=device)
     pat = sa.Pattern(**w.pattern_fields(), random_table=tab,
-                     skipped_in_denominator=w.skipped_in_denominator)
+                     skipped_in_denominator=w.skipped_in_denominator,
+                     row_level_skip=w.row_level_skip)
     plan = sa.Plan(pat, w.B, w.H, w.H_kv, w.N, w.d)
     thresholds = None
     extra = {"plan_compile_ms": round(plan.info["compile_ms"], 2)}
     kept_desc, skipped_pairs = None, 0
-    if w.bsfa:
+    if w.bsfa and w.thresholds == "minus_inf":
+        thresholds = torch.full((w.H,), float("-inf"), dtype=torch.float32, device=device)
+    elif w.bsfa:
         Qc, Kc, _, _ = workloads.calibration_inputs(w, device=device)
-        # the statistics pass is the same for the denominator variant (it
-        # changes what a skipped block contributes, not the decision)
+        # the statistics pass is the same for the rule's variants (they change
+        # what a skipped or dropped block contributes, not the block decision)
         thresholds = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
         del Qc, Kc
+    if w.bsfa:
         mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=device)
         stat = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.float32, device=device)
         plan.prefill(Q, K, V, thresholds=thresholds, block_mask=mask, block_stat=stat)
@@ -477,7 +481,7 @@ def cpu_oracle_rate(w, seconds, sample_seed=0, device_tensors=None, thresholds=N
         t0 = time.perf_counter()
         res = oracle.prefill(opat, Qh, Kh, Vh, thresholds=thresholds, rows=rows, nthreads=cores,
                              keep_in_denominator=bool(w.skipped_in_denominator),
-                             want_blocks=bool(w.bsfa))
+                             row_level=bool(w.row_level_skip), want_blocks=bool(w.bsfa))
         t_total += time.perf_counter() - t0
         for b, h, t, r in tiles:
             if w.bsfa:
@@ -504,6 +508,8 @@ def oracle_thresholds(w, tiles_per_head=4, nthreads=0):
     import numpy as np
     import oracle
     from block_sparse_attention_29_b200 import workloads
+    if w.thresholds == "minus_inf":
+        return np.full(w.H, -np.inf), "of -inf (every block kept)"
     Qc, Kc, _, tab = workloads.calibration_inputs(w, device="cpu")
     opat = oracle.Pattern(**w.pattern_fields(), random_table=tab)
     T = -(-w.N // w.block_q)
@@ -520,10 +526,12 @@ def oracle_thresholds(w, tiles_per_head=4, nthreads=0):
 HEADLINE = "bsfa_causal"
 # Timed after the headline in the same run: the other four configurations of
 # the metric (tiny static pattern, Mistral window, Longformer/BigBird, index-set
-# gather), then the extensions (the block-skip variant, dilated window, window
-# decode, top-K decode).
+# gather), then the block-skip workload with thresholds of -inf (nothing
+# skipped: what the rule saves is measured against it), then the extensions (the
+# rule's two variants, dilated window, window decode, top-K decode).
 SECONDARY = ("mistral_swa", "longformer_bigbird", "gather_decode", "tiny_static",
-             "bsfa_denominator", "dilated_swa", "window_decode", "topk_decode")
+             "bsfa_causal_noskip", "bsfa_denominator", "bsfa_row_level", "dilated_swa",
+             "window_decode", "topk_decode")
 SECONDARY_MIN_S = 0.3   # each secondary workload's timed region lasts at least this long
 
 
@@ -730,6 +738,10 @@ def main():
             Ss = None
             torch.cuda.empty_cache()
         out["secondary"]["workloads"] = table
+        if "bsfa_causal_noskip" in table:
+            # the rule's saving: the same inputs with nothing skipped, over the headline
+            out["secondary"]["block_skip_speedup"] = round(
+                table["bsfa_causal_noskip"]["ms_per_step"] / out["ms_per_step"], 4)
         out["secondary"]["workloads_note"] = (
             "each timed like the headline (CUDA events per step, L2 flushed before every step, "
             "clocks sampled during its own timed region); end-to-end and CPU baseline are "
@@ -760,7 +772,9 @@ def config_of(w, world):
     pat = {k: v for k, v in w.pattern_fields().items() if v and not (k == "dilation" and v == 1)}
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.H_kv, "N": w.N, "d": w.d,
             "pattern": pat, "block_skip_rule": bool(w.bsfa),
+            **({"thresholds": w.thresholds} if w.bsfa else {}),
             **({"skipped_keys_in_denominator": True} if w.skipped_in_denominator else {}),
+            **({"row_level_skip": True} if w.row_level_skip else {}),
             "per_rank": "one replica per GPU", "l2": "256 MiB flush before every step"}
 
 

@@ -65,6 +65,7 @@ class Pattern:
     scale: float = 0.0
     dilation: int = 1   # window taps this far apart (dilated/strided window); 1 = contiguous
     skipped_in_denominator: int = 0   # block-skip variant: skipped keys stay in the denominator
+    row_level_skip: int = 0   # block-skip rule, per-query reading: rows drop full blocks by their own max
 
     def to_c(self, thresholds_ptr: int = 0):
         tab = None
@@ -74,7 +75,7 @@ class Pattern:
                        self.block_k, self.random_block, self.n_random if tab is not None else 0,
                        tab.ctypes.data if tab is not None else None,
                        thresholds_ptr or None, self.scale, self.dilation,
-                       self.skipped_in_denominator)
+                       self.skipped_in_denominator, self.row_level_skip)
         return st, tab   # the caller keeps `tab` alive while the struct is used
 
 

@@ -40,7 +40,7 @@ class SaPattern(ctypes.Structure):
                 ("random_block", ctypes.c_int32), ("n_random", ctypes.c_int32),
                 ("random_table", ctypes.c_void_p), ("thresholds", ctypes.c_void_p),
                 ("scale", ctypes.c_float), ("dilation", ctypes.c_int32),
-                ("skipped_in_denominator", ctypes.c_int32)]
+                ("skipped_in_denominator", ctypes.c_int32), ("row_level_skip", ctypes.c_int32)]
 
 
 class SaPlanInfo(ctypes.Structure):

@@ -126,6 +126,10 @@ int check_shapes(const sa_pattern_t* pat, int B, int H, int Hkv, int N, int d) {
   if (pat->n_random > 0 && pat->random_table && (pat->random_block <= 0 || pat->random_block % kTileK))
     return set_error(SA_ERR_UNSUPPORTED, "random_block = %d must be a positive multiple of 64",
                      pat->random_block);
+  if (pat->row_level_skip && pat->skipped_in_denominator)
+    return set_error(SA_ERR_UNSUPPORTED,
+                     "the row-level block-skip reading is not combined with skipped keys kept "
+                     "in the denominator");
   if (N >= (1 << 28)) return set_error(SA_ERR_UNSUPPORTED, "N = %d too large", N);
   const int dil = pat->dilation > 1 ? pat->dilation : 1;
   const int64_t units = int64_t(B) * dil * H * ((N / dil + kTileQ - 1) / kTileQ);
@@ -192,7 +196,7 @@ std::string cache_key(const sa_pattern_t* p, int B, int H, int Hkv, int N, int d
   auto put = [&k](const void* src, size_t n) { k.append(static_cast<const char*>(src), n); };
   const int32_t f[] = {p->causal, p->window, p->n_global, p->block_local, p->block_q,
                        p->block_k, p->random_block, p->n_random, p->dilation > 1 ? p->dilation : 1,
-                       p->skipped_in_denominator ? 1 : 0,
+                       p->skipped_in_denominator ? 1 : 0, p->row_level_skip ? 1 : 0,
                        B, H, Hkv, N, d, dev};
   put(f, sizeof f);
   put(&p->scale, sizeof p->scale);
@@ -245,6 +249,7 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
   p->random_block = plan->pat.random_block;
   p->n_random = plan->d_rtab ? plan->pat.n_random : 0;
   p->skip_denominator = plan->pat.skipped_in_denominator ? 1 : 0;
+  p->row_level = plan->pat.row_level_skip ? 1 : 0;
   const float scale = plan->pat.scale != 0.f ? plan->pat.scale : 1.0f / sqrtf(float(plan->d));
   p->scale = scale;
   p->scale_log2 = scale * 1.4426950408889634f;
@@ -298,10 +303,12 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
   if (rc) return rc;
   const int dil = pat->dilation > 1 ? pat->dilation : 1;
   if (kernel == SA_KERNEL_PAIRED_HEADS &&
-      (dil > 1 || pat->skipped_in_denominator || !pair_kernel_fits(d, H, H_kv, cp.H_pat)))
+      (dil > 1 || pat->skipped_in_denominator || pat->row_level_skip ||
+       !pair_kernel_fits(d, H, H_kv, cp.H_pat)))
     return set_error(SA_ERR_UNSUPPORTED,
                      "the paired-head kernel needs d = 128, an even number of query heads per "
-                     "K/V head, no random table, no dilation and skipped keys out of G");
+                     "K/V head, no random table, no dilation, skipped keys out of G and the "
+                     "tile-level block-skip rule");
 
   sa_plan_t* plan = new sa_plan_t;
   plan->pat = *pat;

@@ -60,6 +60,7 @@ struct PrefillParams {
   int gate;        // 1: statistics + decision per block (rule or stats pass)
   int stats_only;  // 1: no PV, no output (statistics pass)
   int skip_denominator;  // 1: a skipped block's exp terms still enter m and l
+  int row_level;   // 1: rows also drop full blocks whose own maximum is below the threshold
   int want_stats;  // 1: block statistics needed (stat_out or gate)
   float scale;       // logit scale
   float scale_log2;  // scale * log2(e)

@@ -170,6 +170,7 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   p.random_block = pat->random_block;
   p.n_random = rnd ? pat->n_random : 0;
   p.skip_denominator = pat->skipped_in_denominator ? 1 : 0;
+  p.row_level = pat->row_level_skip ? 1 : 0;
   const float scale = pat->scale != 0.f ? pat->scale : 1.0f / sqrtf(float(d));
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;

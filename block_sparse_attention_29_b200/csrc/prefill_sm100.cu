@@ -488,8 +488,12 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
         }
       }
 
+      // Row-level reading of the rule: a row whose own maximum over a full
+      // block is below the threshold drops the block (P = 0 in its row, no
+      // contribution to its max or sum) while the tile keeps it for other rows.
+      const bool row_drop = p.row_level && p.gate && keep && !partial && (mx * p.scale < tau);
       // Online softmax in the log2 domain with a lazily updated max.
-      const float mx2 = mx * p.scale_log2;
+      const float mx2 = row_drop ? -INFINITY : mx * p.scale_log2;
       const float m_new = fmaxf(m, mx2);
       const bool need = m_new > m + kRescaleLog2 || (m == -INFINITY && m_new != -INFINITY);
       float alpha = 1.f;
@@ -522,7 +526,8 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       // of them to an FMA-pipe polynomial was measured slower: this loop is
       // bound by instruction issue, not by the MUFU pipe.
       const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
-      const uint64_t nmb = f2_pack(-mb, -mb);
+      // a dropped row's exponent arguments are all -inf: p = 0
+      const uint64_t nmb = row_drop ? f2_pack(-INFINITY, -INFINITY) : f2_pack(-mb, -mb);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
 #pragma unroll

@@ -27,6 +27,10 @@ Workloads (names used by tests and bench):
                       each query's 2048 highest-scoring keys (dynamic top-K)
   bsfa_denominator    bsfa_causal's inputs and thresholds with the rule's variant that
                       keeps skipped blocks' keys in the softmax denominator
+  bsfa_causal_noskip  bsfa_causal's inputs with thresholds of -inf (every block computed
+                      and kept: the baseline of the rule's savings)
+  bsfa_row_level      bsfa_causal's inputs and thresholds with the row-level reading of
+                      the rule (rows also drop kept blocks below the threshold)
 """
 from __future__ import annotations
 
@@ -57,6 +61,11 @@ class PrefillWorkload:
     seed: int = 0
     dilation: int = 1
     skipped_in_denominator: int = 0   # block-skip variant (product pattern field)
+    row_level_skip: int = 0           # block-skip rule, per-query reading (product pattern field)
+    # "calibrated": per-head thresholds from the calibration draw; "minus_inf":
+    # thresholds of -inf (the rule computes and keeps every block: the run the
+    # rule's savings are measured against)
+    thresholds: str = "calibrated"
     extra: dict = field(default_factory=dict)
 
     def pattern_fields(self):
@@ -128,6 +137,12 @@ WORKLOADS = {
     "bsfa_denominator": PrefillWorkload("bsfa_denominator", B=1, H=32, H_kv=8, N=32768, d=128,
                                         causal=1, block_q=128, block_k=64, bsfa=True,
                                         skipped_in_denominator=1, seed=3000),
+    "bsfa_causal_noskip": PrefillWorkload("bsfa_causal_noskip", B=1, H=32, H_kv=8, N=32768,
+                                          d=128, causal=1, block_q=128, block_k=64, bsfa=True,
+                                          thresholds="minus_inf", seed=3000),
+    "bsfa_row_level": PrefillWorkload("bsfa_row_level", B=1, H=32, H_kv=8, N=32768, d=128,
+                                      causal=1, block_q=128, block_k=64, bsfa=True,
+                                      row_level_skip=1, seed=3000),
     "dilated_swa": PrefillWorkload("dilated_swa", B=1, H=32, H_kv=8, N=32768, d=128, causal=1,
                                    window=2048, dilation=8, block_q=128, block_k=64, seed=7000),
 }

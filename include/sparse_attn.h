@@ -115,6 +115,17 @@ typedef struct {
                                       load and no PV for it, but its exp terms enter
                                       l and the running max); 0 = they leave G_i.
                                       Single-head kernel only.                          */
+    int32_t row_level_skip;        /* block-skip rule, per-query reading ("Block Sparse
+                                      Flash Attention", paper summary: each query's
+                                      scores decide which value blocks matter): 1 = on
+                                      top of the tile decision, each row drops a full
+                                      block of its tile whose maximum over that row's
+                                      own scaled logits is below the threshold (its
+                                      keys leave that row's G_i).  The V load and PV are
+                                      skipped when every row drops the block, which is
+                                      the tile rule's decision.  0 = tile rule only.
+                                      Not combined with skipped_in_denominator;
+                                      single-head kernel only.                          */
 } sa_pattern_t;
 
 /* A compiled pattern: per-(head, 128-row query tile) lists of 64-key blocks

@@ -96,6 +96,73 @@ def test_bsfa_skipped_keys_in_denominator(product, oracle_mod, cuda, d):
     assert torch.all(lse >= lse0 - 1e-4)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_bsfa_row_level_matches_oracle(product, oracle_mod, cuda, d):
+    """Row-level reading of the rule (each row drops a full block whose maximum
+    over its own logits is below the threshold).  The block masks are the tile
+    rule's (compared as above).  Rows with no (row, block) maximum within 1e-3
+    of the threshold must match the oracle; a row with such pairs must match
+    the oracle replaying one of the combinations of decisions on them."""
+    import itertools
+    w = _small(d=d)
+    Qc, Kc, _, _ = calibration_inputs(w, device="cpu")
+    opat = oracle_mod.Pattern(**w.pattern_fields())
+    full_c, stat_c, _ = oracle_mod.block_stats(opat, Qc, Kc)
+    tau = oracle_mod.calibrate_thresholds(full_c, stat_c).astype(np.float32).astype(np.float64)
+    Q, K, V = _tensors(w, cuda)
+    plan = product.Plan(product.Pattern(**w.pattern_fields(), row_level_skip=1), w.B, w.H,
+                        w.H_kv, w.N, w.d)
+    tau_d = torch.tensor(tau, dtype=torch.float32, device=cuda)
+    mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
+    lse = torch.empty((w.B, w.H, w.N), device=cuda)
+    O = plan.prefill(Q, K, V, thresholds=tau_d, lse=lse, block_mask=mask)
+    O_tile = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N,
+                          w.d).prefill(Q, K, V, thresholds=tau_d)
+    product.check_device_error()
+    Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
+    _, _, om, ost, _ = oracle_mod.prefill(opat, Qh, Kh, Vh, thresholds=tau, want_blocks=True)
+    n, n_near, override = compare_masks(mask.cpu().numpy(), om, ost, tau)
+    Or, lr, _, _, _, rstat = oracle_mod.prefill(opat, Qh, Kh, Vh, thresholds=tau, row_level=True,
+                                                override=override, want_blocks=True,
+                                                want_row_stats=True)
+    n_kb = plan.n_kb
+    tau_r = np.repeat(tau, w.N)[:, None]   # per flat row [H*N] (B = 1)
+    near = np.isfinite(rstat) & (np.abs(rstat - tau_r) <= NEAR_BAND)
+    near_rows = np.nonzero(near.any(axis=1))[0]
+    ok = np.ones(w.B * w.H * w.N, bool)
+    ok[near_rows] = False
+    Og = O.cpu().reshape(-1, w.d)
+    lg = lse.cpu().reshape(-1)
+    Or, lr = Or.reshape(-1, w.d), lr.reshape(-1)
+    assert_close(Og[torch.from_numpy(ok)], Or[ok])
+    assert_close(lg[torch.from_numpy(ok)], lr[ok], what="lse")
+    for r in near_rows:
+        kbs = np.nonzero(near[r])[0]
+        assert len(kbs) <= 3, "too many near-threshold blocks in one row"
+        b, h, i = 0, int(r // w.N), int(r % w.N)
+        best = np.inf
+        for combo in itertools.product((0, 1), repeat=len(kbs)):
+            ro = np.full((1, n_kb), -1, np.int8)
+            ro[0, kbs] = combo
+            Oc, _ = oracle_mod.prefill(opat, Qh, Kh, Vh, thresholds=tau, row_level=True,
+                                       override=override, rows=np.array([[b, h, i]], np.int32),
+                                       row_override=ro)
+            best = min(best, float(np.abs(Og[r].double().numpy() - Oc[0]).max()))
+        assert best <= 1e-2, (r, kbs, best)
+    # the reading is in effect: rows that drop a block the tile keeps differ
+    assert not torch.equal(O, O_tile)
+
+
+def test_bsfa_row_level_refusals(product, cuda):
+    w = _small()
+    with pytest.raises(product.SparseAttnError):
+        product.Plan(product.Pattern(**w.pattern_fields(), row_level_skip=1), w.B, w.H, w.H_kv,
+                     w.N, w.d, kernel=product.KERNEL_PAIRED_HEADS)
+    with pytest.raises(product.SparseAttnError):
+        product.Plan(product.Pattern(**w.pattern_fields(), row_level_skip=1,
+                                     skipped_in_denominator=1), w.B, w.H, w.H_kv, w.N, w.d)
+
+
 def test_bsfa_denominator_variant_is_single_head_only(product, cuda):
     w = _small()
     with pytest.raises(product.SparseAttnError):
@@ -203,8 +270,9 @@ def test_bsfa_full_size_sampled(product, oracle_mod, cuda, kernel, record_proper
     tau_o, tau_o32, om, ost, ofull = _oracle_whole_heads(oracle_mod, w, heads)
     plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
                         kernel=kernel)
-    Qc, Kc, _, _ = calibration_inputs(w, device=cuda)
-    tau_d = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)
+    # inputs drawn once on the host (the oracle's copy and the device's are the same bytes)
+    Qc, Kc, _, _ = calibration_inputs(w, device="cpu")
+    tau_d = plan.calibrate(plan.block_stats(Qc.to(cuda), Kc.to(cuda)), 0.5)
     del Qc, Kc
     tau_gpu = tau_d.cpu().numpy().astype(np.float64)
     hs = list(heads)
@@ -213,7 +281,7 @@ def test_bsfa_full_size_sampled(product, oracle_mod, cuda, kernel, record_proper
     tau_run = tau_gpu.copy()
     tau_run[hs] = tau_o32[hs]
     tau_d = torch.tensor(tau_run, dtype=torch.float32, device=cuda)
-    Q, K, V, _ = prefill_inputs(w, device=cuda)
+    Q, K, V = (x.to(cuda) for x in prefill_inputs(w, device="cpu")[:3])
     mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
     stat = torch.empty((w.B, w.H, plan.T, plan.n_kb), device=cuda)
     O = plan.prefill(Q, K, V, thresholds=tau_d, block_mask=mask, block_stat=stat)
