@@ -42,7 +42,7 @@ import numpy as np
 from ._lib import (EXPORTS, LIB_PATH, SA_ERR_DEVICE_INDEX, SA_ERR_INVALID_ARG, SA_ERR_TIMEOUT,
                    SA_ERR_UNSUPPORTED, SA_OK, SaPattern, SaPlanInfo, SparseAttnError, check, lib)
 
-__all__ = ["Pattern", "Plan", "KERNEL_AUTO", "KERNEL_SINGLE_HEAD", "KERNEL_PAIRED_HEADS",
+__all__ = ["Pattern", "Plan", "KERNEL_AUTO", "KERNEL_SINGLE_HEAD",
            "sparse_attn_prefill", "sparse_attn_prefill_noalloc",
            "sparse_attn_gather", "sparse_attn_decode_window", "window_slot",
            "sparse_attn_decode_topk", "decode_topk_workspace_bytes", "compile_pattern",
@@ -105,15 +105,12 @@ def _check_tensor(name, t, shape, dtype):
 
 KERNEL_AUTO = 0            # the kernel measured fastest for the shape (single-head today)
 KERNEL_SINGLE_HEAD = 1     # the single-head kernel
-KERNEL_PAIRED_HEADS = 2    # the paired-head kernel (d=128, even GQA group, no random table)
 
 
 class Plan:
     """A compiled pattern for Q [B][H][N][d], K/V [B][H_kv][N][d].
 
-    ``kernel``: KERNEL_AUTO, KERNEL_SINGLE_HEAD or KERNEL_PAIRED_HEADS
-    (sparse_attn_plan_create_ex); ``info["paired_heads"]`` tells which kernel
-    the plan runs on."""
+    ``kernel``: KERNEL_AUTO or KERNEL_SINGLE_HEAD (sparse_attn_plan_create_ex)."""
 
     def __init__(self, pattern: Pattern, B: int, H: int, H_kv: int, N: int, d: int,
                  kernel: int = KERNEL_AUTO):

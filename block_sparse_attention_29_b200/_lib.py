@@ -48,8 +48,7 @@ class SaPlanInfo(ctypes.Structure):
     _fields_ = [("T_q", ctypes.c_int32), ("n_kb", ctypes.c_int32),
                 ("n_units", ctypes.c_int64), ("blocks", ctypes.c_int64),
                 ("blocks_full", ctypes.c_int64), ("blocks_desc", ctypes.c_int64),
-                ("pairs", ctypes.c_int64), ("compile_ms", ctypes.c_double),
-                ("paired_heads", ctypes.c_int32)]
+                ("pairs", ctypes.c_int64), ("compile_ms", ctypes.c_double)]
 
 
 class SparseAttnError(RuntimeError):

@@ -19,9 +19,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libsparse_attn.so")
-SOURCES = ["api.cu", "pattern_compiler.cu", "prefill_sm100.cu", "prefill_pair_sm100.cu",
-           "gather_sm100.cu", "topk_sm100.cu", "calibrate.cu",
-           "noalloc.cu"]
+SOURCES = ["api.cu", "pattern_compiler.cu", "prefill_sm100.cu", "gather_sm100.cu",
+           "topk_sm100.cu", "calibrate.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + CSRC, "-I" + INCLUDE]

@@ -148,7 +148,6 @@ struct sa_plan {
   int T = 0, n_kb = 0, H_pat = 0;
   int dil = 1;                 // dilation: the plan's lists cover one of dil residue classes
   int n_units = 0;
-  bool pair = false;           // paired-head kernel (units are head pairs)
   int32_t* d_row_ptr = nullptr;
   int32_t* d_entries = nullptr;
   int32_t* d_units = nullptr;
@@ -233,7 +232,6 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
   p->rtab = plan->d_rtab;
   p->thresholds = thresholds;
   p->n_units = plan->n_units;
-  p->pair = plan->pair ? 1 : 0;
   p->B = plan->B;
   p->H = plan->H;
   p->Hkv = plan->Hkv;
@@ -291,8 +289,7 @@ int sparse_attn_plan_create(const sa_pattern_t* pat, int B, int H, int H_kv, int
 int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, int N, int d,
                                int kernel, sa_plan_t** out) {
   if (!out) return set_error(SA_ERR_INVALID_ARG, "out is NULL");
-  if (kernel != SA_KERNEL_AUTO && kernel != SA_KERNEL_SINGLE_HEAD &&
-      kernel != SA_KERNEL_PAIRED_HEADS)
+  if (kernel != SA_KERNEL_AUTO && kernel != SA_KERNEL_SINGLE_HEAD)
     return set_error(SA_ERR_INVALID_ARG, "kernel = %d (not an SA_KERNEL_* value)", kernel);
   *out = nullptr;
   int rc = check_shapes(pat, B, H, H_kv, N, d);
@@ -302,14 +299,6 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
   rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
   if (rc) return rc;
   const int dil = pat->dilation > 1 ? pat->dilation : 1;
-  if (kernel == SA_KERNEL_PAIRED_HEADS &&
-      (dil > 1 || pat->skipped_in_denominator || pat->row_level_skip ||
-       !pair_kernel_fits(d, H, H_kv, cp.H_pat)))
-    return set_error(SA_ERR_UNSUPPORTED,
-                     "the paired-head kernel needs d = 128, an even number of query heads per "
-                     "K/V head, no random table, no dilation, skipped keys out of G and the "
-                     "tile-level block-skip rule");
-
   sa_plan_t* plan = new sa_plan_t;
   plan->pat = *pat;
   plan->pat.random_table = nullptr;
@@ -355,11 +344,9 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
     plan->info.blocks_desc = int64_t(cd.kb.size()) * int64_t(Bd) * (cd.H_pat == 1 ? H : 1);
   }
 
-  plan->pair = kernel == SA_KERNEL_PAIRED_HEADS;
-  plan->info.paired_heads = plan->pair ? 1 : 0;
-  plan->n_units = Bd * cp.T * (plan->pair ? H / 2 : H);
+  plan->n_units = Bd * cp.T * H;
   std::vector<int32_t> units;
-  build_units(cp, Bd, H, H_kv, N / dil, d, plan->pair, &units);
+  build_units(cp, Bd, H, H_kv, N / dil, d, &units);
 
   rc = upload(&plan->d_row_ptr, cp.row_ptr.data(), cp.row_ptr.size());
   if (!rc) rc = upload(&plan->d_entries, entries.data(), entries.size());

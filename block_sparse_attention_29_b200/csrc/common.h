@@ -44,8 +44,7 @@ struct PrefillParams {
   float* stat_out;    // [B][H][T][n_kb] or null
   const int32_t* row_ptr;   // [H_pat*T + 1]
   const int32_t* entries;   // block lists
-  const int32_t* units;     // work order: unit = (b'*H + h)*T + t, or with pair = 1
-                            // (b'*(H/2) + hp)*T + t for the heads 2hp and 2hp + 1;
+  const int32_t* units;     // work order: unit = (b'*H + h)*T + t with
                             // b' = b*dil + residue class (b' = b without dilation)
   int* sched;               // [2] work-queue counters (next unit, CTAs done); zero
                             // between launches (the last CTA of a launch resets them)
@@ -56,7 +55,6 @@ struct PrefillParams {
                                          // N: positions per residue class (N/dil)
   int dil;         // dilation: query/key position m of class r is row m*dil + r
   int causal, window, n_global, block_local, random_block, n_random;
-  int pair;        // 1: units are head pairs (paired-head kernel), 0: single heads
   int gate;        // 1: statistics + decision per block (rule or stats pass)
   int stats_only;  // 1: no PV, no output (statistics pass)
   int skip_denominator;  // 1: a skipped block's exp terms still enter m and l
@@ -68,15 +66,6 @@ struct PrefillParams {
 };
 
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream);
-int launch_prefill_pair(const PrefillParams& p, int d, cudaStream_t stream);
-
-// The paired-head kernel runs two query heads of one K/V group per work unit
-// and shares every K and V tile between them.  It needs d = 128, an even
-// number of query heads per K/V head and block lists shared by all heads (no
-// per-head random table).
-inline bool pair_kernel_fits(int d, int H, int H_kv, int H_pat) {
-  return d == 128 && H_pat == 1 && H % H_kv == 0 && (H / H_kv) % 2 == 0;
-}
 
 // 4-D bf16 TMA map over a [BH][N][d] tensor seen as [BH][N/dil][dil][d]:
 // coordinates (x, r, m, slice) address row m*dil + r; box {64, 1, rows, 1},
@@ -153,18 +142,16 @@ int check_shapes(const sa_pattern_t* pat, int B, int H, int Hkv, int N, int d);
 // half a CTA's share first (longest first), the rest tile-major or
 // K/V-group-major (see kv_bytes), the query heads of a group adjacent.
 // kv_bytes: size of K plus V; above 64 MiB (half of L2) the order is
-// K/V-group-major, below tile-major.  H counts the heads of a unit's index
-// (head pairs for the paired-head kernel); ctas is the number of CTAs that
-// share the queue.
+// K/V-group-major, below tile-major.  ctas is the number of CTAs that share
+// the queue.
 void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_bytes, int ctas,
                  std::vector<int32_t>* units);
 
-// Work units of a launch in queue order for the kernel that `pair` selects.
-inline void build_units(const CompiledPattern& cp, int B, int H, int H_kv, int N, int d, bool pair,
+// Work units of a prefill launch in queue order (two CTAs per SM share the queue).
+inline void build_units(const CompiledPattern& cp, int B, int H, int H_kv, int N, int d,
                         std::vector<int32_t>* units) {
   const int64_t kv_bytes = int64_t(B) * H_kv * N * d * 2 * 2;
-  if (pair) order_units(cp, B, H / 2, H_kv, kv_bytes, 148, units);
-  else order_units(cp, B, H, H_kv, kv_bytes, 296, units);
+  order_units(cp, B, H, H_kv, kv_bytes, 296, units);
 }
 
 }  // namespace sa

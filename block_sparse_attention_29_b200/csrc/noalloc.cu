@@ -91,11 +91,10 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
   if (rc) return rc;
   const int T = cp.T;
-  const bool pair = false;   // the single-head kernel (the default of the plan API)
   const int dil = pat->dilation > 1 ? pat->dilation : 1;
   if (dil > 1 && pat->thresholds)
     return set_error(SA_ERR_UNSUPPORTED, "a dilated window takes no block-skip thresholds");
-  const int64_t n_units = int64_t(B) * dil * (pair ? H / 2 : H) * T;
+  const int64_t n_units = int64_t(B) * dil * H * T;
   const int nrb = rnd ? (N + pat->random_block - 1) / pat->random_block : 0;
   const size_t b_row = round256(cp.row_ptr.size() * 4);
   const size_t b_ent = round256(std::max<size_t>(cp.kb.size(), 1) * 4);
@@ -112,7 +111,7 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   std::vector<int32_t> entries(cp.kb.size());
   for (size_t e = 0; e < cp.kb.size(); ++e) entries[e] = entry_pack(cp.kb[e], !cp.full[e]);
   std::vector<int32_t> units;
-  build_units(cp, B * dil, H, H_kv, N / dil, d, pair, &units);
+  build_units(cp, B * dil, H, H_kv, N / dil, d, &units);
 
   unsigned char* base = nullptr;
   rc = scratch_address(&base);
@@ -154,7 +153,6 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
   p.rtab = d_rtab;
   p.thresholds = pat->thresholds;
   p.n_units = int(n_units);
-  p.pair = pair ? 1 : 0;
   p.B = B;
   p.H = H;
   p.Hkv = H_kv;

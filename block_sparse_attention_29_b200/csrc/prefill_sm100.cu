@@ -26,12 +26,13 @@
 // them) and each CTA's producer claims the next one with an atomic counter
 // when it has room, so CTAs that get cheap units take more of them.
 //
-// TMEM columns: two S buffers at [0, 64) and [64, 128), O at [128, 128 + d).
-// Block k uses S buffer k % 2; its P (bf16 pairs) is written over the first
-// 32 columns of that buffer once the logits are in registers, and the PV of
-// block k reads it there.  The QK^T of block k+1 runs while the softmax works
-// on block k, also when block k is skipped by the rule, so a run of skipped
-// blocks costs the softmax's statistic alone per block.
+// TMEM columns: NS S buffers of 64 columns at [0, 64 NS) (NS = 2 at d = 128,
+// 3 at d = 64, where O is half as wide), O at [64 NS, 64 NS + d).  Block k
+// uses S buffer k % NS; its P (bf16 pairs) is written over the first 32
+// columns of that buffer once the logits are in registers, and the PV of block
+// k reads it there.  The QK^T of the next NS - 1 blocks runs while the softmax
+// works on block k, also when block k is skipped by the rule, so a run of
+// skipped blocks costs the softmax's statistic alone per block.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -45,8 +46,7 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;
-constexpr int kTmemS = 0;     // two S buffers of 64 fp32 columns, at kTmemS + 64 b
-constexpr int kTmemO = 128;   // O accumulator: d fp32 columns
+constexpr int kTmemS = 0;     // S buffers of 64 fp32 columns, at kTmemS + 64 b
 constexpr uint32_t kSoftmaxBar = 1;    // named barrier of the softmax warpgroup
 constexpr uint32_t kSoftmaxWarps = 4;
 constexpr float kRescaleLog2 = 8.0f;   // lazy rescale: keep a stale max up to 2^8
@@ -55,6 +55,13 @@ constexpr uint32_t kUnitRing = 4;       // depth of the work-unit ring
 // each softmax warp
 constexpr uint32_t kUnitConsumers = 1 + 1 + 4;
 constexpr uint32_t kDecRing = 4;        // depth of the gate-decision ring
+// PV completions are tracked on a ring of kODone barriers (PV number n on
+// barrier n % kODone, phase n / kODone).  A softmax warp waits on PV number L
+// only after the S of its current block has landed, and S(k) is issued after
+// block k - NS is handled, so every PV older than L - NS + 1 is complete: the
+// parity wait on L's barrier cannot mistake an older phase for L's while
+// kODone >= NS + 1.
+constexpr uint32_t kODone = 4;
 
 // where-codes recorded with SA_ERR_TIMEOUT
 enum { W_PROD_Q = 1, W_PROD_K, W_MMA_Q, W_MMA_SFREE, W_MMA_K, W_MMA_VEMPTY, W_MMA_DEC,
@@ -66,6 +73,13 @@ struct Cfg {
   static constexpr int KS = D == 128 ? 2 : 3;   // K ring depth
   static constexpr int VS = D == 128 ? 2 : 3;   // V ring depth
   static constexpr int CH = D / 64;             // 64-column (128-byte) chunks per row
+  static constexpr int NS = D == 128 ? 2 : 3;   // S buffers in TMEM
+  // d = 64 (BigBird-style patterns): warps whose rows see no key of a random
+  // block skip it; at d = 128 the plain loop is kept (measured faster there)
+  static constexpr bool kSkipInvisible = D == 64;
+  static_assert(kODone >= NS + 1, "PV-completion ring too shallow for NS S buffers");
+  static constexpr int TMEM_O = kTmemS + 64 * NS;   // O accumulator: d fp32 columns
+  static_assert(TMEM_O + D <= kTmemCols, "TMEM budget");
   static constexpr int Q_BYTES = kTileQ * D * 2;
   static constexpr int KV_BYTES = kTileK * D * 2;
   static constexpr int OFF_Q = 0;
@@ -87,16 +101,16 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[3], k_empty[3];
   uint64_t v_full[3], v_empty[3];
-  uint64_t s_full[2];                   // per S buffer: S of the block written
-  uint64_t p_ready[2];                  // per block parity: P written (or block skipped)
+  uint64_t s_full[3];                   // per S buffer: S of the block written
+  uint64_t p_ready[3];                  // per S buffer: P written (or block skipped)
   uint64_t dec_full[4], dec_empty[4];   // gate decisions, softmax -> V loader
-  uint64_t o_done[2];
+  uint64_t o_done[4];
   uint64_t drain;
   uint64_t u_full[4], u_empty[4];   // work-unit ring (producer -> MMA + softmax)
   uint32_t tmem_base;
   int abort;
-  uint32_t flags[2];   // per block parity: 1 = block kept, 0 = skipped
-  float red[2][4];     // per block parity: warp maxima for the tile maximum
+  uint32_t flags[3];   // per S buffer: 1 = block kept, 0 = skipped
+  float red[3][4];     // per S buffer: warp maxima for the tile maximum
   Unit unit_slot[4];   // decoded work unit; n = -1 once the queue is exhausted
   uint32_t dec_val[4]; // decision ring: 1 = keep, 0 = skip
 };
@@ -302,11 +316,11 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
     uint32_t idle = 0;
     while (npv < u.n) {
       bool progress = false;
-      // S for block ns.
-      if (ns < u.n && ns <= npv + 1) {
+      // S for block ns (its buffer's previous block, ns - NS, handled).
+      if (ns < u.n && ns <= npv + C::NS - 1) {
         const uint32_t st = kc % C::KS;
         if (mbar_try_wait(smem_u32(&bars->k_full[st]), (kc / C::KS) & 1)) {
-          const uint32_t sb = (g0 + ns) & 1;
+          const uint32_t sb = (g0 + ns) % C::NS;
           const uint32_t kbase = sK + st * C::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -326,8 +340,8 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
       }
       // P hand-off of block nr.
       if (nr < ns) {
-        const uint32_t gk = g0 + nr, fb = gk & 1;
-        if (mbar_try_wait(smem_u32(&bars->p_ready[fb]), (gk >> 1) & 1)) {
+        const uint32_t gk = g0 + nr, fb = gk % C::NS;
+        if (mbar_try_wait(smem_u32(&bars->p_ready[fb]), (gk / C::NS) & 1)) {
           tc_fence_after();
           if (flags[fb]) keep_bits |= 1u << (nr & 31);
           else keep_bits &= ~(1u << (nr & 31));
@@ -345,15 +359,15 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
           if (mbar_try_wait(smem_u32(&bars->v_full[vs]), (pvc / C::VS) & 1)) {
             tc_fence_after();
             const uint32_t vbase = sV + vs * C::KV_BYTES;
-            const uint32_t pcol = kTmemS + 64 * ((g0 + npv) & 1);   // P over block npv's S
+            const uint32_t pcol = kTmemS + 64 * ((g0 + npv) % C::NS);   // P over block npv's S
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
               const uint64_t db = make_sdesc(vbase + kk * (16 * 128), kTileK * 128, 1024);
-              umma_ts(tmem + kTmemO, tmem + pcol + kk * 8, db, idesc_o,
+              umma_ts(tmem + C::TMEM_O, tmem + pcol + kk * 8, db, idesc_o,
                       (first_pv && kk == 0) ? 0u : 1u);
             }
             tc_commit(smem_u32(&bars->v_empty[vs]));
-            tc_commit(smem_u32(&bars->o_done[pvc & 1]));
+            tc_commit(smem_u32(&bars->o_done[pvc % kODone]));
             ++pvc;
             ++npv;
             first_pv = false;
@@ -390,6 +404,7 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
 template <int D>
 __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, int warp,
                              int lane) {
+  using C = Cfg<D>;
   volatile int* abort_flag = &bars->abort;
   volatile uint32_t* flags = bars->flags;
   const int q4 = warp & 3;              // TMEM lane quadrant of this warp
@@ -415,13 +430,18 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
     const RowVis rv = row_vis(p, load_row_random(p, u.h, i), i);
 
     for (int k = 0; k < u.n; ++k) {
-      const uint32_t fb = g & 1;   // per-block-parity flag / decision slot
+      const uint32_t fb = g % C::NS;   // this block's S buffer (and flag / statistic slot)
       const int e = e_next;
       if (k + 1 < u.n) e_next = __ldg(p.entries + u.beg + k + 1);
       const int kb = e >> 1;
       const bool partial = e & 1;
       uint64_t vis = ~0ull;
       if (partial) vis = vis_bits(p, rv, u.h, i, kb);
+      // A warp none of whose rows sees a key of this (partial) block -- the
+      // other half of the tile of a random block drawn for 64 query rows --
+      // neither reads S nor computes exponentials: its rows' P is zero.
+      const bool none =
+          C::kSkipInvisible && p.n_random > 0 && partial && __all_sync(0xffffffffu, vis == 0ull);
       // The leader claims this block's decision-ring slot now, while S is
       // still being computed (the V loader frees slots as it reads them).
       bool slot_ok = true;
@@ -431,11 +451,12 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       // S of this block is in S buffer fb; the MMA thread computes the next
       // block's S into the other buffer meanwhile.
       const uint32_t tS = tmem + lane_base + kTmemS + 64 * fb;
-      if (!wait_bounded(smem_u32(&bars->s_full[fb]), (g >> 1) & 1, abort_flag, p.err, W_SM_S))
+      if (!wait_bounded(smem_u32(&bars->s_full[fb]), (g / C::NS) & 1, abort_flag, p.err, W_SM_S))
         return;
       tc_fence_after();
       float x[64];
-      {
+      float mx = -INFINITY;
+      if (!none) {
         uint32_t r0[32], r1[32];
         tmem_ld32(tS, r0);
         tmem_ld32(tS + 32, r1);
@@ -445,9 +466,9 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
           x[c] = __uint_as_float(r0[c]);
           x[32 + c] = __uint_as_float(r1[c]);
         }
+        if (partial && vis != ~0ull) apply_mask(vis, x);
+        mx = row_max64(x);
       }
-      if (partial && vis != ~0ull) apply_mask(vis, x);
-      const float mx = row_max64(x);
 
       bool keep = true;
       if (p.want_stats) {
@@ -505,14 +526,14 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       if (kept > 0 && __any_sync(0xffffffffu, need)) {
         // O += P V of the previous kept block must be complete before O is rescaled.
         const uint32_t last = pv_total - 1;
-        if (!wait_bounded(smem_u32(&bars->o_done[last & 1]), (last >> 1) & 1, abort_flag, p.err,
-                          W_SM_O))
+        if (!wait_bounded(smem_u32(&bars->o_done[last % kODone]), (last / kODone) & 1, abort_flag,
+                          p.err, W_SM_O))
           return;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          const uint32_t ta = tmem + lane_base + kTmemO + c * 32;
+          const uint32_t ta = tmem + lane_base + C::TMEM_O + c * 32;
           tmem_ld32(ta, o);
           tmem_wait_ld();
 #pragma unroll
@@ -530,16 +551,19 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       const uint64_t nmb = row_drop ? f2_pack(-INFINITY, -INFINITY) : f2_pack(-mb, -mb);
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
+      if (none) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float a0, a1, p0, p1;
-        f2_unpack(f2_fma(f2_pack(x[2 * c], x[2 * c + 1]), sl2, nmb), a0, a1);
-        p0 = ex2(a0);
-        p1 = ex2(a1);
-        acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
-        pk[c] = pack_bf16x2(p0, p1);
-      }
-      {
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float a0, a1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(x[2 * c], x[2 * c + 1]), sl2, nmb), a0, a1);
+          p0 = ex2(a0);
+          p1 = ex2(a1);
+          acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+        }
         float s0, s1;
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
         l += s0 + s1;
@@ -567,15 +591,15 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
     uint16_t* orow_ptr = p.O + orow * D;
     if (kept > 0) {
       const uint32_t last = pv_total - 1;
-      if (!wait_bounded(smem_u32(&bars->o_done[last & 1]), (last >> 1) & 1, abort_flag, p.err,
-                        W_SM_EPI))
+      if (!wait_bounded(smem_u32(&bars->o_done[last % kODone]), (last / kODone) & 1, abort_flag,
+                        p.err, W_SM_EPI))
         return;
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + kTmemO + c * 32, o);
+        tmem_ld32(tmem + lane_base + C::TMEM_O + c * 32, o);
         tmem_wait_ld();
         if (row_ok) {
           uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c * 32);
@@ -617,11 +641,11 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
       mbar_init(smem_u32(&bars->v_full[s]), 1);
       mbar_init(smem_u32(&bars->v_empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(smem_u32(&bars->s_full[b]), 1);
       mbar_init(smem_u32(&bars->p_ready[b]), kSoftmaxWarps);
-      mbar_init(smem_u32(&bars->o_done[b]), 1);
     }
+    for (uint32_t b = 0; b < kODone; ++b) mbar_init(smem_u32(&bars->o_done[b]), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     for (uint32_t r = 0; r < kDecRing; ++r) {
       mbar_init(smem_u32(&bars->dec_full[r]), 1);
@@ -632,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
       mbar_init(smem_u32(&bars->u_empty[r]), kUnitConsumers);
     }
     bars->abort = 0;
-    bars->flags[0] = bars->flags[1] = 0;
+    bars->flags[0] = bars->flags[1] = bars->flags[2] = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -679,7 +703,6 @@ bool g_attr_set[2][64] = {{false}};
 }  // namespace
 
 int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream) {
-  if (p.pair) return launch_prefill_pair(p, d, stream);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");

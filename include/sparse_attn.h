@@ -143,20 +143,13 @@ typedef struct {
     int64_t blocks_desc;    /* listed blocks at the descriptor's block_q x block_k      */
     int64_t pairs;          /* sum over (b, h, i) of |G_i| of the static pattern        */
     double compile_ms;      /* host time spent compiling the pattern                    */
-    int32_t paired_heads;   /* 1: the plan runs on the paired-head kernel (two query
-                               heads of one K/V head per work unit, d = 128, an even
-                               number of query heads per K/V head, block lists shared
-                               by all heads); 0: the single-head kernel             */
 } sa_plan_info_t;
 
 /* Kernel choice for sparse_attn_plan_create_ex. */
 enum {
     SA_KERNEL_AUTO = 0,          /* the kernel measured fastest for the plan's shape on
-                                    B200: currently the single-head kernel everywhere   */
-    SA_KERNEL_SINGLE_HEAD = 1,   /* the single-head kernel                                */
-    SA_KERNEL_PAIRED_HEADS = 2   /* the paired-head kernel (d = 128, an even number of
-                                    query heads per K/V head, no random table);
-                                    SA_ERR_UNSUPPORTED elsewhere                         */
+                                    B200: the single-head kernel                         */
+    SA_KERNEL_SINGLE_HEAD = 1    /* the single-head kernel                                */
 };
 
 /* Compile `pat` for Q [B][H][N][d], K/V [B][H_kv][N][d].  Host work plus
@@ -170,10 +163,7 @@ enum {
 int sparse_attn_plan_create(const sa_pattern_t *pat, int B, int H, int H_kv, int N, int d,
                             sa_plan_t **out);
 /* Same as sparse_attn_plan_create with an explicit kernel choice (SA_KERNEL_*;
- * other values: SA_ERR_INVALID_ARG; SA_KERNEL_PAIRED_HEADS for a plan it does
- * not apply to: SA_ERR_UNSUPPORTED).  Both kernels compute the same result;
- * they differ only in rounding order (the paired-head kernel updates the
- * running maximum once per two key blocks). */
+ * other values: SA_ERR_INVALID_ARG). */
 int sparse_attn_plan_create_ex(const sa_pattern_t *pat, int B, int H, int H_kv, int N, int d,
                                int kernel, sa_plan_t **out);
 int sparse_attn_plan_info(const sa_plan_t *plan, sa_plan_info_t *info);

@@ -176,10 +176,7 @@ def test_plan_refusals_on_host(product):
     assert plan(causal=1, window=8, dilation=7) == product.SA_ERR_UNSUPPORTED      # 7 does not divide 600
     assert plan(causal=1, window=8, dilation=3, n_global=2) == product.SA_ERR_UNSUPPORTED
     assert plan(causal=1, window=0, dilation=3) == product.SA_ERR_INVALID_ARG
-    assert plan(causal=1, window=8, dilation=3,
-                kernel=product.KERNEL_PAIRED_HEADS) == product.SA_ERR_UNSUPPORTED
-    assert plan(causal=1, skipped_in_denominator=1,
-                kernel=product.KERNEL_PAIRED_HEADS) == product.SA_ERR_UNSUPPORTED
+    assert plan(causal=1, kernel=2) == product.SA_ERR_INVALID_ARG   # no longer a kernel
     assert plan(causal=1, kernel=7) == product.SA_ERR_INVALID_ARG
 
 

@@ -27,9 +27,8 @@ def _tensors(w, device):
     return Q.to(device), K.to(device), V.to(device)
 
 
-@pytest.mark.parametrize("d,kernel", [(128, 0), (128, 2), (64, 0)],
-                         ids=["d128", "d128-paired", "d64"])
-def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d, kernel):
+@pytest.mark.parametrize("d", [128, 64])
+def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d):
     w = _small(d=d)
     Qc, Kc, Vc, _ = calibration_inputs(w, device="cpu")
     opat = oracle_mod.Pattern(**w.pattern_fields())
@@ -38,9 +37,7 @@ def test_bsfa_small_matches_oracle(product, oracle_mod, cuda, d, kernel):
     # the same (rounded) threshold values
     tau = oracle_mod.calibrate_thresholds(full_c, stat_c).astype(np.float32).astype(np.float64)
     Q, K, V = _tensors(w, cuda)
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
-                        kernel=kernel)
-    assert plan.info["paired_heads"] == int(kernel == 2)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
     tau_d = torch.tensor(tau, dtype=torch.float32, device=cuda)
     mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
     stat = torch.full((w.B, w.H, plan.T, plan.n_kb), float("-inf"), device=cuda)
@@ -156,26 +153,14 @@ def test_bsfa_row_level_matches_oracle(product, oracle_mod, cuda, d):
 def test_bsfa_row_level_refusals(product, cuda):
     w = _small()
     with pytest.raises(product.SparseAttnError):
-        product.Plan(product.Pattern(**w.pattern_fields(), row_level_skip=1), w.B, w.H, w.H_kv,
-                     w.N, w.d, kernel=product.KERNEL_PAIRED_HEADS)
-    with pytest.raises(product.SparseAttnError):
         product.Plan(product.Pattern(**w.pattern_fields(), row_level_skip=1,
                                      skipped_in_denominator=1), w.B, w.H, w.H_kv, w.N, w.d)
 
 
-def test_bsfa_denominator_variant_is_single_head_only(product, cuda):
-    w = _small()
-    with pytest.raises(product.SparseAttnError):
-        product.Plan(product.Pattern(**w.pattern_fields(), skipped_in_denominator=1), w.B, w.H,
-                     w.H_kv, w.N, w.d, kernel=product.KERNEL_PAIRED_HEADS)
-
-
-@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
-def test_bsfa_extreme_thresholds(product, oracle_mod, cuda, kernel):
+def test_bsfa_extreme_thresholds(product, oracle_mod, cuda):
     w = _small(N=768, H=2, Hkv=1)
     Q, K, V = _tensors(w, cuda)
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
-                        kernel=kernel)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
     mask = torch.empty((w.B, w.H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
     # -inf: nothing skipped, equals the static causal path bit for bit
     O_static = plan.prefill(Q, K, V)
@@ -203,13 +188,11 @@ def test_bsfa_extreme_thresholds(product, oracle_mod, cuda, kernel):
     assert_close(O_pinf, Or)
 
 
-@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
-def test_device_calibration_matches_oracle(product, oracle_mod, cuda, kernel):
+def test_device_calibration_matches_oracle(product, oracle_mod, cuda):
     """Statistics pass + per-head rank selection on the GPU == oracle calibration."""
     w = _small(N=1024, H=4, Hkv=2)
     Qc, Kc, _, _ = calibration_inputs(w, device="cpu")
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
-                        kernel=kernel)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
     stat = plan.block_stats(Qc.to(cuda), Kc.to(cuda))
     tau_gpu = plan.calibrate(stat, 0.5).cpu().numpy()
     opat = oracle_mod.Pattern(**w.pattern_fields())
@@ -256,8 +239,7 @@ def _oracle_whole_heads(oracle_mod, w, heads):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
-def test_bsfa_full_size_sampled(product, oracle_mod, cuda, kernel, record_property):
+def test_bsfa_full_size_sampled(product, oracle_mod, cuda, record_property):
     """bsfa_causal at N=32768.  Every block of every head: the decision is the
     rule applied to the kernel's statistic.  Every tile of FULL_HEADS: the
     device calibration equals the oracle's, and with the oracle's thresholds the
@@ -268,8 +250,7 @@ def test_bsfa_full_size_sampled(product, oracle_mod, cuda, kernel, record_proper
     heads = FULL_HEADS
     assert heads[-1] == w.H - 1
     tau_o, tau_o32, om, ost, ofull = _oracle_whole_heads(oracle_mod, w, heads)
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
-                        kernel=kernel)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
     # inputs drawn once on the host (the oracle's copy and the device's are the same bytes)
     Qc, Kc, _, _ = calibration_inputs(w, device="cpu")
     tau_d = plan.calibrate(plan.block_stats(Qc.to(cuda), Kc.to(cuda)), 0.5)
@@ -329,16 +310,14 @@ def test_bsfa_full_size_sampled(product, oracle_mod, cuda, kernel, record_proper
     assert_close(O.cpu()[sel], Or)
 
 
-@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
 @pytest.mark.parametrize("tau_kind", ["calibrated", "plus_inf"])
-def test_bsfa_repeated_launches_stable(product, oracle_mod, cuda, tau_kind, kernel):
+def test_bsfa_repeated_launches_stable(product, oracle_mod, cuda, tau_kind):
     """Many launches of the rule without block outputs (the timing of the
     benchmark loop), including pairs of key blocks that both heads skip: no
     pipeline wait may run out and every launch gives the same bytes."""
     w = _small(N=4096, H=8, Hkv=2)
     Q, K, V = _tensors(w, cuda)
-    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d,
-                        kernel=kernel)
+    plan = product.Plan(product.Pattern(**w.pattern_fields()), w.B, w.H, w.H_kv, w.N, w.d)
     if tau_kind == "calibrated":
         Qc, Kc, _, _ = calibration_inputs(w, device=cuda)
         tau = plan.calibrate(plan.block_stats(Qc, Kc), 0.5)

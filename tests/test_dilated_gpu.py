@@ -107,9 +107,6 @@ def test_dilated_window_refusals(product, cuda):
         product.Plan(product.Pattern(causal=1, window=8, dilation=7), B, H, Hkv, N, d)
     with pytest.raises(product.SparseAttnError):      # combined with global tokens
         product.Plan(product.Pattern(causal=1, window=8, dilation=3, n_global=2), B, H, Hkv, N, d)
-    with pytest.raises(product.SparseAttnError):      # paired-head kernel
-        product.Plan(product.Pattern(causal=1, window=8, dilation=3), B, H, Hkv, N, d,
-                     kernel=product.KERNEL_PAIRED_HEADS)
     plan = product.Plan(product.Pattern(causal=1, window=8, dilation=3), B, H, Hkv, N, d)
     thr = torch.zeros(H, dtype=torch.float32, device=cuda)
     with pytest.raises(product.SparseAttnError):      # block-skip rule

@@ -21,20 +21,11 @@ def _rand(shape, seed, device):
     return torch.randn(shape, generator=g).to(torch.bfloat16).to(device)
 
 
-def _paired_applies(H, Hkv, d, pat):
-    return d == 128 and (H // Hkv) % 2 == 0 and pat.get("random_table") is None
-
-
-def _run_case(product, oracle_mod, cuda, B, H, Hkv, N, d, seed, kernel=0, **pat):
+def _run_case(product, oracle_mod, cuda, B, H, Hkv, N, d, seed, **pat):
     Q = _rand((B, H, N, d), seed, cuda)
     K = _rand((B, Hkv, N, d), seed + 1, cuda)
     V = _rand((B, Hkv, N, d), seed + 2, cuda)
-    if kernel == product.KERNEL_PAIRED_HEADS and not _paired_applies(H, Hkv, d, pat):
-        with pytest.raises(product.SparseAttnError):
-            product.Plan(product.Pattern(**pat), B, H, Hkv, N, d, kernel=kernel)
-        return None, None
-    plan = product.Plan(product.Pattern(**pat), B, H, Hkv, N, d, kernel=kernel)
-    assert plan.info["paired_heads"] == int(kernel == product.KERNEL_PAIRED_HEADS)
+    plan = product.Plan(product.Pattern(**pat), B, H, Hkv, N, d)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=cuda)
     mask = torch.empty((B, H, plan.T, plan.n_kb), dtype=torch.uint8, device=cuda)
     O = plan.prefill(Q, K, V, lse=lse, block_mask=mask)
@@ -69,38 +60,19 @@ CASES = [
     # |out| reaches 3 and bf16 output rounding alone (half-ulp 0.0078 there) plus
     # bf16 P rounding exceed the 1e-2 budget
     dict(B=1, H=2, Hkv=2, N=200, d=128, causal=1, window=5, scale=0.125),
-    # paired-head kernel: lists of odd and even lengths (a lone last block),
-    # partial blocks on both sides of a pair, several head pairs per K/V head
+    # lists of odd and even lengths, partial blocks on both window edges,
+    # several query heads per K/V head
     dict(B=2, H=8, Hkv=2, N=700, d=128, causal=0, window=150, n_global=7),
     dict(B=1, H=4, Hkv=2, N=1100, d=128, causal=1, window=520, n_global=3),
     dict(B=1, H=2, Hkv=1, N=1300, d=128, causal=1, block_local=192),
 ]
 
 
-@pytest.mark.parametrize("kernel", [0, 2], ids=["auto", "paired"])
 @pytest.mark.parametrize("case", range(len(CASES)))
-def test_prefill_small(product, oracle_mod, cuda, case, kernel):
+def test_prefill_small(product, oracle_mod, cuda, case):
     c = dict(CASES[case])
     _run_case(product, oracle_mod, cuda, c.pop("B"), c.pop("H"), c.pop("Hkv"), c.pop("N"),
-              c.pop("d"), 100 + 7 * case, kernel=kernel, **c)
-
-
-def test_paired_and_single_head_kernels_agree(product, cuda):
-    """The two kernels compute the same attention; only the rounding order of
-    the running maximum differs."""
-    B, H, Hkv, N, d = 1, 8, 2, 2048, 128
-    Q, K, V = _rand((B, H, N, d), 11, cuda), _rand((B, Hkv, N, d), 12, cuda), _rand(
-        (B, Hkv, N, d), 13, cuda)
-    pat = product.Pattern(causal=1, window=700, n_global=5)
-    p2 = product.Plan(pat, B, H, Hkv, N, d, kernel=product.KERNEL_PAIRED_HEADS)
-    p1 = product.Plan(pat, B, H, Hkv, N, d, kernel=product.KERNEL_SINGLE_HEAD)
-    assert p2.info["paired_heads"] == 1 and p1.info["paired_heads"] == 0
-    l1, l2 = (torch.empty((B, H, N), device=cuda) for _ in range(2))
-    O1 = p1.prefill(Q, K, V, lse=l1)
-    O2 = p2.prefill(Q, K, V, lse=l2)
-    product.check_device_error()
-    assert_close(O2, O1.float().cpu())
-    assert (l1 - l2).abs().max().item() < 1e-4
+              c.pop("d"), 100 + 7 * case, **c)
 
 
 def test_prefill_random_blocks(product, oracle_mod, cuda):
@@ -146,15 +118,12 @@ def _sample_rows(B, H, N, n_random, seed):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,kernel", [("mistral_swa", 0), ("mistral_swa", 2),
-                                         ("longformer_bigbird", 0), ("dilated_swa", 0)],
-                         ids=["mistral_swa", "mistral_swa-paired", "longformer_bigbird",
-                              "dilated_swa"])
-def test_prefill_full_size_sampled(product, oracle_mod, cuda, name, kernel):
+@pytest.mark.parametrize("name", ["mistral_swa", "longformer_bigbird", "dilated_swa"])
+def test_prefill_full_size_sampled(product, oracle_mod, cuda, name):
     w = WORKLOADS[name]
     Q, K, V, tab = prefill_inputs(w, device=cuda)
     plan = product.Plan(product.Pattern(**w.pattern_fields(), random_table=tab), w.B, w.H, w.H_kv,
-                        w.N, w.d, kernel=kernel)
+                        w.N, w.d)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=cuda)
     O = plan.prefill(Q, K, V, lse=lse)
     product.check_device_error()
