@@ -316,7 +316,7 @@ def setup_window_decode(w, device, torch, sa, workloads):
     return dict(step=step, e2e_step=e2e_step, h2d=h2d, d2h=d2h, flops=flops, exact_flops=flops,
                 dense_flops=flops, algo_bytes=algo_bytes,
                 extra={"rows_per_query": n_rows, "cache_slots": n_rows},
-                kernel="gather_group_kernel", kernel_files=["gather_sm100.cu"],
+                kernel="window_group_kernel", kernel_files=["gather_sm100.cu", "ptx.cuh"],
                 metric="window decode GB/s", unit="GB/s", bound="hbm",
                 tensors=(Q, K, V, pos, O), pos=pos)
 
