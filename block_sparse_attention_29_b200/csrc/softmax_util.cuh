@@ -53,13 +53,17 @@ __device__ __forceinline__ RowRandom load_row_random(const PrefillParams& p, int
 // kb*64 + c).  Every primitive is one index range per row (random blocks cover
 // whole 64-key blocks), so the union is built from ranges; the causal cap and
 // the sequence end are applied last.  Same predicate as the pattern compiler.
-// The per-row part (window start, cap, the row's random blocks as the first
-// 64-key block of their range) is computed once per work unit by row_vis, so
-// a block's mask costs a few range masks and compares and no division.
+// The per-row part (the global, window and block-local ranges, the cap, the
+// row's random blocks as the first 64-key block of their range) is computed
+// once per work unit by row_vis, so a block's mask reads no pattern field and
+// costs a few compares and range masks, no division.
 struct RowVis {
   int all;              // the row sees every key below cap_hi (global row, or no primitive)
-  int win_lo;           // window keys [win_lo, win_lo + window length)
+  int glob_hi;          // global keys [0, glob_hi) (0 when there are none)
+  int win_lo, win_hi;   // window keys [win_lo, win_hi) (empty when there is no window)
+  int bl_lo, bl_hi;     // block-local keys [bl_lo, bl_hi) (empty when off)
   int cap_hi;           // causal cap and sequence end: keys < cap_hi (0 for rows past N)
+  int rb64;             // 64-key blocks per random block (0 when there are none)
   int rlo[kRowRandom];  // the row's first random blocks, as their first 64-key block
 };
 
@@ -67,43 +71,48 @@ __device__ __forceinline__ RowVis row_vis(const PrefillParams& p, const RowRando
   RowVis v;
   const bool any_prim = p.window > 0 || p.n_global > 0 || p.block_local > 0 || p.n_random > 0;
   v.all = (!any_prim || i < p.n_global) ? 1 : 0;
-  v.win_lo = p.causal ? i - p.window + 1 : i - p.window / 2;
+  v.glob_hi = p.n_global;
+  if (p.window > 0) {
+    v.win_lo = p.causal ? i - p.window + 1 : i - p.window / 2;
+    v.win_hi = v.win_lo + (p.causal ? p.window : 2 * (p.window / 2) + 1);
+  } else {
+    v.win_lo = v.win_hi = 0;
+  }
+  if (p.block_local > 0) {
+    v.bl_lo = (i / p.block_local) * p.block_local;
+    v.bl_hi = v.bl_lo + p.block_local;
+  } else {
+    v.bl_lo = v.bl_hi = 0;
+  }
   v.cap_hi = i >= p.N ? 0 : (p.causal ? i + 1 : p.N);
-  const int rb64 = p.random_block / kTileK;
+  v.rb64 = p.n_random > 0 ? p.random_block / kTileK : 0;
 #pragma unroll
-  for (int r = 0; r < kRowRandom; ++r) v.rlo[r] = r < rr.n ? rr.v[r] * rb64 : -(1 << 30);
+  for (int r = 0; r < kRowRandom; ++r) v.rlo[r] = r < rr.n ? rr.v[r] * v.rb64 : -(1 << 30);
   return v;
 }
 
+// Visible keys of row i inside block kb from the row's precomputed ranges:
+// random blocks first (a listed random block is visible in full), then the
+// union of the global, window and block-local ranges, capped.
 __device__ __forceinline__ uint64_t vis_bits(const PrefillParams& p, const RowVis& v, int h,
                                              int i, int kb) {
   const int j0 = kb * kTileK;
-  uint64_t m = ~0ull;
-  if (!v.all) {
-    m = range_bits(0, p.n_global - j0);
-    if (p.window > 0) {
-      const int len = p.causal ? p.window : 2 * (p.window / 2) + 1;
-      m |= range_bits(v.win_lo - j0, v.win_lo + len - j0);
-    }
-    if (p.block_local > 0) {
-      const int lo = (i / p.block_local) * p.block_local;
-      m |= range_bits(lo - j0, lo + p.block_local - j0);
-    }
-    if (p.n_random > 0) {
-      const unsigned rb64 = static_cast<unsigned>(p.random_block / kTileK);
-      bool rnd = false;
+  const uint64_t cap = range_bits(0, v.cap_hi - j0);
+  if (v.all) return cap;
+  const unsigned rb64 = static_cast<unsigned>(v.rb64);
+  bool rnd = false;
 #pragma unroll
-      for (int r = 0; r < kRowRandom; ++r) rnd |= static_cast<unsigned>(kb - v.rlo[r]) < rb64;
-      if (p.n_random > kRowRandom && i < p.N) {   // longer lists: read from the table
-        const int nrb = (p.N + p.random_block - 1) / p.random_block;
-        const int32_t* row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
-        for (int r = kRowRandom; r < p.n_random; ++r)
-          rnd |= static_cast<unsigned>(kb - __ldg(row + r) * static_cast<int>(rb64)) < rb64;
-      }
-      if (rnd) m = ~0ull;
-    }
+  for (int r = 0; r < kRowRandom; ++r) rnd |= static_cast<unsigned>(kb - v.rlo[r]) < rb64;
+  if (p.n_random > kRowRandom && i < p.N) {   // longer lists: read from the table
+    const int nrb = (p.N + p.random_block - 1) / p.random_block;
+    const int32_t* row = p.rtab + ((int64_t)h * nrb + i / p.random_block) * p.n_random;
+    for (int r = kRowRandom; r < p.n_random; ++r)
+      rnd |= static_cast<unsigned>(kb - __ldg(row + r) * static_cast<int>(rb64)) < rb64;
   }
-  return m & range_bits(0, v.cap_hi - j0);
+  if (rnd) return cap;
+  const uint64_t m = range_bits(0, v.glob_hi - j0) | range_bits(v.win_lo - j0, v.win_hi - j0) |
+                     range_bits(v.bl_lo - j0, v.bl_hi - j0);
+  return m & cap;
 }
 
 // x[OFF + c] = -inf where bit c of the visibility mask is clear.
