@@ -188,9 +188,13 @@ def setup_prefill(w, device, torch, sa, workloads):
     pat = sa.Pattern(**w.pattern_fields(), random_table=tab,
                      skipped_in_denominator=w.skipped_in_denominator,
                      row_level_skip=w.row_level_skip)
-    plan = sa.Plan(pat, w.B, w.H, w.H_kv, w.N, w.d)
+    plan = sa.Plan(pat, w.B, w.H, w.H_kv, w.N, w.d, max_unit_blocks=w.max_unit_blocks)
     thresholds = None
     extra = {"plan_compile_ms": round(plan.info["compile_ms"], 2)}
+    if plan.info["split_tiles"]:
+        # tiles cut into pieces (one more kernel per step merges them)
+        extra["split_tiles"] = plan.info["split_tiles"]
+        extra["queue_units"] = plan.info["queue_units"]
     kept_desc, skipped_pairs = None, 0
     if w.bsfa and w.thresholds == "minus_inf":
         thresholds = torch.full((w.H,), float("-inf"), dtype=torch.float32, device=device)
@@ -249,6 +253,7 @@ def setup_prefill(w, device, torch, sa, workloads):
     return dict(step=step, e2e_step=lambda s: e2e_step(host, dev_bufs, s), h2d=h2d, d2h=d2h,
                 flops=computed, exact_flops=exact, dense_flops=dense, algo_bytes=algo_bytes,
                 extra=extra, kernel="prefill_kernel",
+                launches_per_step=2 if plan.info["split_tiles"] else 1,
                 kernel_files=["prefill_sm100.cu", "softmax_util.cuh", "ptx.cuh", "common.h",
                               "pattern_compiler.cu"],
                 metric="effective TFLOP/s (computed blocks)", unit="TFLOP/s", bound="tensor",
@@ -528,10 +533,11 @@ HEADLINE = "bsfa_causal"
 # the metric (tiny static pattern, Mistral window, Longformer/BigBird, index-set
 # gather), then the block-skip workload with thresholds of -inf (nothing
 # skipped: what the rule saves is measured against it), then the extensions (the
-# rule's two variants, dilated window, window decode, top-K decode).
+# rule's two variants, dilated window, window decode, top-K decode, split tiles
+# forced and automatic).
 SECONDARY = ("mistral_swa", "longformer_bigbird", "gather_decode", "tiny_static",
              "bsfa_causal_noskip", "bsfa_denominator", "bsfa_row_level", "dilated_swa",
-             "window_decode", "topk_decode")
+             "window_decode", "topk_decode", "longformer_split", "bigbird_two_heads")
 SECONDARY_MIN_S = 0.3   # each secondary workload's timed region lasts at least this long
 
 

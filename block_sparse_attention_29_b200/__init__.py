@@ -40,7 +40,8 @@ from typing import Optional
 import numpy as np
 
 from ._lib import (EXPORTS, LIB_PATH, SA_ERR_DEVICE_INDEX, SA_ERR_INVALID_ARG, SA_ERR_TIMEOUT,
-                   SA_ERR_UNSUPPORTED, SA_OK, SaPattern, SaPlanInfo, SparseAttnError, check, lib)
+                   SA_ERR_UNSUPPORTED, SA_OK, SaPattern, SaPlanInfo, SaPlanOptions, SparseAttnError,
+                   check, lib)
 
 __all__ = ["Pattern", "Plan", "KERNEL_AUTO", "KERNEL_SINGLE_HEAD",
            "sparse_attn_prefill", "sparse_attn_prefill_noalloc",
@@ -110,15 +111,19 @@ KERNEL_SINGLE_HEAD = 1     # the single-head kernel
 class Plan:
     """A compiled pattern for Q [B][H][N][d], K/V [B][H_kv][N][d].
 
-    ``kernel``: KERNEL_AUTO or KERNEL_SINGLE_HEAD (sparse_attn_plan_create_ex)."""
+    ``kernel``: KERNEL_AUTO or KERNEL_SINGLE_HEAD; ``max_unit_blocks``: 0 splits a
+    tile whose list exceeds one CTA's share of the launch, > 0 cuts every block
+    list longer than that into pieces, < 0 splits nothing
+    (sparse_attn_plan_create_opts)."""
 
     def __init__(self, pattern: Pattern, B: int, H: int, H_kv: int, N: int, d: int,
-                 kernel: int = KERNEL_AUTO):
+                 kernel: int = KERNEL_AUTO, max_unit_blocks: int = 0):
         self.pattern, self.B, self.H, self.H_kv, self.N, self.d = pattern, B, H, H_kv, N, d
         st, _tab = pattern.to_c()
         h = ctypes.c_void_p()
-        check(lib().sparse_attn_plan_create_ex(ctypes.byref(st), B, H, H_kv, N, d, kernel,
-                                               ctypes.byref(h)))
+        opts = SaPlanOptions(kernel, max_unit_blocks)
+        check(lib().sparse_attn_plan_create_opts(ctypes.byref(st), B, H, H_kv, N, d,
+                                                 ctypes.byref(opts), ctypes.byref(h)))
         self._h = h
         info = SaPlanInfo()
         check(lib().sparse_attn_plan_info(self._h, ctypes.byref(info)))
@@ -342,6 +347,25 @@ def compile_pattern(pattern: Pattern, H: int, N: int, tile_q: int = 128, tile_k:
                                         kb.ctypes.data, full.ctypes.data, cnt.ctypes.data))
     n = n.value
     return row_ptr, kb[:n], full[:n].astype(bool), cnt[:n], hp.value, T.value
+
+
+def work_order(pattern: Pattern, B: int, H: int, H_kv: int, N: int, d: int,
+               max_unit_blocks: int = 0):
+    """Host work order of a plan's prefill queue: (units, pieces [n][4], split [n][4])
+    as numpy int32 arrays (sparse_attn_work_order)."""
+    st, _tab = pattern.to_c()
+    nu, npc, ns = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    L = lib()
+    check(L.sparse_attn_work_order(ctypes.byref(st), B, H, H_kv, N, d, max_unit_blocks,
+                                   ctypes.byref(nu), ctypes.byref(npc), ctypes.byref(ns),
+                                   None, None, None))
+    units = np.zeros(max(nu.value, 1), np.int32)
+    pieces = np.zeros((max(npc.value, 1), 4), np.int32)
+    split = np.zeros((max(ns.value, 1), 4), np.int32)
+    check(L.sparse_attn_work_order(ctypes.byref(st), B, H, H_kv, N, d, max_unit_blocks,
+                                   ctypes.byref(nu), ctypes.byref(npc), ctypes.byref(ns),
+                                   units.ctypes.data, pieces.ctypes.data, split.ctypes.data))
+    return units[:nu.value], pieces[:npc.value], split[:ns.value]
 
 
 def check_device_error(stream=None) -> None:

@@ -22,11 +22,12 @@ SA_ERR_DEVICE_INDEX = 6
 
 # Every function the header declares (tests check the library exports them all).
 EXPORTS = (
-    "sparse_attn_plan_create", "sparse_attn_plan_create_ex", "sparse_attn_plan_info",
+    "sparse_attn_plan_create", "sparse_attn_plan_create_ex", "sparse_attn_plan_create_opts",
+    "sparse_attn_plan_info",
     "sparse_attn_plan_destroy",
     "sparse_attn_prefill_plan", "sparse_attn_prefill", "sparse_attn_block_stats",
     "sparse_attn_calibrate", "sparse_attn_gather", "sparse_attn_decode_window",
-    "sparse_attn_window_slot", "sparse_attn_compile_pattern",
+    "sparse_attn_window_slot", "sparse_attn_compile_pattern", "sparse_attn_work_order",
     "sparse_attn_check_device_error", "sparse_attn_last_error", "sparse_attn_prefill_noalloc",
     "sparse_attn_decode_topk", "sparse_attn_decode_topk_workspace",
 )
@@ -48,7 +49,14 @@ class SaPlanInfo(ctypes.Structure):
     _fields_ = [("T_q", ctypes.c_int32), ("n_kb", ctypes.c_int32),
                 ("n_units", ctypes.c_int64), ("blocks", ctypes.c_int64),
                 ("blocks_full", ctypes.c_int64), ("blocks_desc", ctypes.c_int64),
-                ("pairs", ctypes.c_int64), ("compile_ms", ctypes.c_double)]
+                ("pairs", ctypes.c_int64), ("compile_ms", ctypes.c_double),
+                ("split_tiles", ctypes.c_int64), ("queue_units", ctypes.c_int64),
+                ("workspace_bytes", ctypes.c_int64)]
+
+
+class SaPlanOptions(ctypes.Structure):
+    """sa_plan_options_t."""
+    _fields_ = [("kernel", ctypes.c_int32), ("max_unit_blocks", ctypes.c_int32)]
 
 
 class SparseAttnError(RuntimeError):
@@ -74,6 +82,9 @@ def lib():
         L.sparse_attn_plan_create.argtypes = [P, i32, i32, i32, i32, i32, ctypes.POINTER(vp)]
         L.sparse_attn_plan_create_ex.argtypes = [P, i32, i32, i32, i32, i32, i32,
                                                  ctypes.POINTER(vp)]
+        L.sparse_attn_plan_create_opts.argtypes = [P, i32, i32, i32, i32, i32,
+                                                   ctypes.POINTER(SaPlanOptions),
+                                                   ctypes.POINTER(vp)]
         L.sparse_attn_plan_info.argtypes = [vp, ctypes.POINTER(SaPlanInfo)]
         L.sparse_attn_plan_destroy.argtypes = [vp]
         L.sparse_attn_plan_destroy.restype = None
@@ -90,6 +101,8 @@ def lib():
         L.sparse_attn_decode_topk_workspace.argtypes = [i32, i32, i32, i32]
         L.sparse_attn_gather.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                          i32, f32, vp, vp]
+        L.sparse_attn_work_order.argtypes = [P, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp,
+                                             vp, vp]
         L.sparse_attn_compile_pattern.argtypes = [P, i32, i32, i32, i32,
                                                   ctypes.POINTER(ctypes.c_int),
                                                   ctypes.POINTER(ctypes.c_int),

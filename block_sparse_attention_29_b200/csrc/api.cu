@@ -151,6 +151,10 @@ struct sa_plan {
   int32_t* d_row_ptr = nullptr;
   int32_t* d_entries = nullptr;
   int32_t* d_units = nullptr;
+  int4* d_pieces = nullptr;    // split-tile pieces (two int4 each, see PrefillParams)
+  int* d_split_cnt = nullptr;  // pieces finished per split tile, zero between launches
+  float* d_part = nullptr;     // pieces' partial results [slot][d + 2][128]
+  int n_split = 0;
   int32_t* d_rtab = nullptr;
   int* d_sched = nullptr;      // work-queue counters, zero between launches
   sa_plan_info_t info{};
@@ -169,6 +173,9 @@ void plan_free(sa_plan_t* p) {
   cudaFree(p->d_row_ptr);
   cudaFree(p->d_entries);
   cudaFree(p->d_units);
+  cudaFree(p->d_pieces);
+  cudaFree(p->d_split_cnt);
+  cudaFree(p->d_part);
   cudaFree(p->d_rtab);
   cudaFree(p->d_sched);
   if (prev >= 0 && prev != p->device) cudaSetDevice(prev);
@@ -228,6 +235,10 @@ int fill_prefill_params(const sa_plan_t* plan, const void* Q, const void* K, con
   p->row_ptr = plan->d_row_ptr;
   p->entries = plan->d_entries;
   p->units = plan->d_units;
+  p->pieces = plan->d_pieces;
+  p->part = plan->d_part;
+  p->split_cnt = plan->d_split_cnt;
+  p->n_split = plan->n_split;
   p->sched = plan->d_sched;
   p->rtab = plan->d_rtab;
   p->thresholds = thresholds;
@@ -262,6 +273,43 @@ extern "C" {
 
 const char* sparse_attn_last_error(void) { return sa::g_msg; }
 
+int sparse_attn_work_order(const sa_pattern_t* pat, int B, int H, int H_kv, int N, int d,
+                           int max_unit_blocks, int64_t* n_units_out, int64_t* n_pieces_out,
+                           int64_t* n_split_out, int32_t* units, int32_t* pieces,
+                           int32_t* split) {
+  int rc = check_shapes(pat, B, H, H_kv, N, d);
+  if (rc) return rc;
+  CompiledPattern cp;
+  rc = compile_pattern(pat, H, N, kTileQ, kTileK, &cp);
+  if (rc) return rc;
+  const int dil = pat->dilation > 1 ? pat->dilation : 1;
+  UnitOrder order;
+  build_units(cp, B * dil, H, H_kv, N / dil, d, max_unit_blocks, &order);
+  if (n_units_out) *n_units_out = int64_t(order.units.size());
+  if (n_pieces_out) *n_pieces_out = int64_t(order.pieces.size());
+  if (n_split_out) *n_split_out = int64_t(order.split.size());
+  if (units) {
+    if ((!pieces && !order.pieces.empty()) || (!split && !order.split.empty()))
+      return set_error(SA_ERR_INVALID_ARG, "pieces and split must be given with units");
+    std::copy(order.units.begin(), order.units.end(), units);
+    for (size_t k = 0; k < order.pieces.size(); ++k) {
+      const Piece& pc = order.pieces[k];
+      pieces[4 * k + 0] = pc.id;
+      pieces[4 * k + 1] = pc.k0;
+      pieces[4 * k + 2] = pc.n;
+      pieces[4 * k + 3] = pc.slot;
+    }
+    for (size_t k = 0; k < order.split.size(); ++k) {
+      const SplitTile& st = order.split[k];
+      split[4 * k + 0] = st.id;
+      split[4 * k + 1] = st.first_slot;
+      split[4 * k + 2] = st.n_pieces;
+      split[4 * k + 3] = 0;
+    }
+  }
+  return SA_OK;
+}
+
 int sparse_attn_compile_pattern(const sa_pattern_t* pat, int H, int N, int tile_q, int tile_k,
                                 int* H_pat_out, int* T_out, int64_t* n_entries_out,
                                 int32_t* row_ptr, int32_t* kb, uint8_t* full, int64_t* cnt) {
@@ -288,7 +336,17 @@ int sparse_attn_plan_create(const sa_pattern_t* pat, int B, int H, int H_kv, int
 
 int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, int N, int d,
                                int kernel, sa_plan_t** out) {
+  sa_plan_options_t o;
+  o.kernel = kernel;
+  o.max_unit_blocks = 0;
+  return sparse_attn_plan_create_opts(pat, B, H, H_kv, N, d, &o, out);
+}
+
+int sparse_attn_plan_create_opts(const sa_pattern_t* pat, int B, int H, int H_kv, int N, int d,
+                                 const sa_plan_options_t* opts, sa_plan_t** out) {
   if (!out) return set_error(SA_ERR_INVALID_ARG, "out is NULL");
+  const int kernel = opts ? opts->kernel : SA_KERNEL_AUTO;
+  const int max_unit_blocks = opts ? opts->max_unit_blocks : 0;
   if (kernel != SA_KERNEL_AUTO && kernel != SA_KERNEL_SINGLE_HEAD)
     return set_error(SA_ERR_INVALID_ARG, "kernel = %d (not an SA_KERNEL_* value)", kernel);
   *out = nullptr;
@@ -344,13 +402,30 @@ int sparse_attn_plan_create_ex(const sa_pattern_t* pat, int B, int H, int H_kv, 
     plan->info.blocks_desc = int64_t(cd.kb.size()) * int64_t(Bd) * (cd.H_pat == 1 ? H : 1);
   }
 
-  plan->n_units = Bd * cp.T * H;
-  std::vector<int32_t> units;
-  build_units(cp, Bd, H, H_kv, N / dil, d, &units);
+  UnitOrder order;
+  build_units(cp, Bd, H, H_kv, N / dil, d, max_unit_blocks, &order);
+  const std::vector<int32_t>& units = order.units;
+  plan->n_units = int(units.size());
+  plan->n_split = int(order.split.size());
+  plan->info.split_tiles = int64_t(order.split.size());
+  plan->info.queue_units = int64_t(units.size());
+  plan->info.workspace_bytes = order.n_slots * piece_slot_floats(d) * int64_t(sizeof(float));
 
   rc = upload(&plan->d_row_ptr, cp.row_ptr.data(), cp.row_ptr.size());
   if (!rc) rc = upload(&plan->d_entries, entries.data(), entries.size());
   if (!rc) rc = upload(&plan->d_units, units.data(), units.size());
+  if (!rc && !order.pieces.empty()) {
+    static_assert(sizeof(Piece) == 2 * sizeof(int4), "a piece is two int4");
+    rc = upload(&plan->d_pieces, reinterpret_cast<const int4*>(order.pieces.data()),
+                2 * order.pieces.size());
+    if (!rc) {
+      const std::vector<int32_t> zeros(order.split.size(), 0);
+      rc = upload(&plan->d_split_cnt, zeros.data(), zeros.size());
+    }
+    if (!rc)
+      rc = upload(&plan->d_part, static_cast<const float*>(nullptr),
+                  size_t(order.n_slots * piece_slot_floats(d)));
+  }
   if (!rc) {
     const int zeros[2] = {0, 0};
     rc = upload(&plan->d_sched, zeros, 2);

@@ -45,7 +45,14 @@ struct PrefillParams {
   const int32_t* row_ptr;   // [H_pat*T + 1]
   const int32_t* entries;   // block lists
   const int32_t* units;     // work order: unit = (b'*H + h)*T + t with
-                            // b' = b*dil + residue class (b' = b without dilation)
+                            // b' = b*dil + residue class (b' = b without dilation);
+                            // a negative entry u is the piece ~u of a split tile
+  const int4* pieces;       // split-tile pieces, two int4 each: {id, k0, n, slot},
+                            // {split tile, its first slot, its pieces, 0}; or null
+  float* part;              // piece workspace [slot][d + 2][128] or null
+  int* split_cnt;           // [n_split] pieces finished per split tile; zero between
+                            // launches (the last CTA of a launch resets them)
+  int n_split;              // split tiles
   int* sched;               // [2] work-queue counters (next unit, CTAs done); zero
                             // between launches (the last CTA of a launch resets them)
   const int32_t* rtab;      // random table [H][n_rb][n_random] or null
@@ -138,20 +145,44 @@ int validate_pattern(const sa_pattern_t* pat, int H, int N);
 // Shapes and the descriptor fields the kernels constrain (head dim, block
 // sizes, random-block granularity, grid and index limits); SA_OK or an error.
 int check_shapes(const sa_pattern_t* pat, int B, int H, int Hkv, int N, int d);
-// Work order of the B*H*T units (unit = (b*H + h)*T + t): units longer than
-// half a CTA's share first (longest first), the rest tile-major or
-// K/V-group-major (see kv_bytes), the query heads of a group adjacent.
-// kv_bytes: size of K plus V; above 64 MiB (half of L2) the order is
-// K/V-group-major, below tile-major.  ctas is the number of CTAs that share
-// the queue.
+// A piece of a split tile: blocks [k0, k0 + n) of tile `id`'s list, whose
+// unnormalised partial result goes to workspace slot `slot`; the tile is split
+// tile `split`, whose n_pieces pieces hold slots [first_slot, first_slot + n_pieces).
+struct Piece {
+  int32_t id, k0, n, slot;
+  int32_t split, first_slot, n_pieces, pad;
+};
+// A split tile: its pieces hold slots [first_slot, first_slot + n_pieces).
+struct SplitTile {
+  int32_t id, first_slot, n_pieces, pad;
+};
+// Work order of a prefill launch.  units[k] >= 0 is a whole tile
+// ((b*H + h)*T + t); units[k] < 0 is pieces[~units[k]].
+struct UnitOrder {
+  std::vector<int32_t> units;
+  std::vector<Piece> pieces;
+  std::vector<SplitTile> split;
+  int64_t n_slots = 0;
+};
+// Work order of the B*H*T tiles: tiles longer than a CTA's share of the work
+// split into pieces (max_unit_blocks: 0 automatic, > 0 the longest list a unit
+// may have, < 0 never; slot_bytes: workspace bytes per piece), units longer than half a
+// CTA's share first (longest first), the rest tile-major or K/V-group-major
+// (see kv_bytes), the query heads of a group adjacent.  kv_bytes: size of K
+// plus V; above 64 MiB (half of L2) the order is K/V-group-major, below
+// tile-major.  ctas is the number of CTAs that share the queue.
 void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_bytes, int ctas,
-                 std::vector<int32_t>* units);
+                 int max_unit_blocks, int64_t slot_bytes, UnitOrder* out);
+
+// Partial-result workspace of one piece: d O columns, then the row maximum
+// (log2 domain) and the row sum, each as 128 consecutive floats (one per row).
+inline int64_t piece_slot_floats(int d) { return int64_t(d + 2) * kTileQ; }
 
 // Work units of a prefill launch in queue order (two CTAs per SM share the queue).
 inline void build_units(const CompiledPattern& cp, int B, int H, int H_kv, int N, int d,
-                        std::vector<int32_t>* units) {
+                        int max_unit_blocks, UnitOrder* order) {
   const int64_t kv_bytes = int64_t(B) * H_kv * N * d * 2 * 2;
-  order_units(cp, B, H, H_kv, kv_bytes, 296, units);
+  order_units(cp, B, H, H_kv, kv_bytes, 296, max_unit_blocks, piece_slot_floats(d) * 4, order);
 }
 
 }  // namespace sa

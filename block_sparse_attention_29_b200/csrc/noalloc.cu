@@ -110,8 +110,10 @@ extern "C" int sparse_attn_prefill_noalloc(const void* Q, const void* K, const v
 
   std::vector<int32_t> entries(cp.kb.size());
   for (size_t e = 0; e < cp.kb.size(); ++e) entries[e] = entry_pack(cp.kb[e], !cp.full[e]);
-  std::vector<int32_t> units;
-  build_units(cp, B * dil, H, H_kv, N / dil, d, &units);
+  // No tile is split here: the pieces' workspace would not fit the scratch.
+  UnitOrder order;
+  build_units(cp, B * dil, H, H_kv, N / dil, d, -1, &order);
+  const std::vector<int32_t>& units = order.units;
 
   unsigned char* base = nullptr;
   rc = scratch_address(&base);

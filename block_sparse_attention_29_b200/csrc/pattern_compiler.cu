@@ -175,47 +175,133 @@ int compile_pattern(const sa_pattern_t* p, int H, int N, int tile_q, int tile_k,
 }
 
 void order_units(const CompiledPattern& cp, int B, int H, int H_kv, int64_t kv_bytes, int ctas,
-                 std::vector<int32_t>* out) {
+                 int max_unit_blocks, int64_t slot_bytes, UnitOrder* out) {
   const int T = cp.T;
   const int64_t n = int64_t(B) * H * T;
-  out->resize(size_t(n));
-  std::vector<int32_t>& units = *out;
-  for (int64_t u = 0; u < n; ++u) units[u] = int32_t(u);
-  auto cost = [&](int32_t u) {
+  auto cost_of = [&](int32_t u) {
     const int t = u % T, h = (u / T) % H;
     const int row = (cp.H_pat > 1 ? h : 0) * T + t;
     return cp.row_ptr[row + 1] - cp.row_ptr[row];
   };
   int64_t total = 0;
-  for (int64_t u = 0; u < n; ++u) total += cost(int32_t(u));
+  std::vector<int32_t> costs;
+  costs.reserve(size_t(n));
+  for (int64_t u = 0; u < n; ++u) {
+    costs.push_back(cost_of(int32_t(u)));
+    total += costs.back();
+  }
   // Units longer than half of one CTA's share of the work would set the tail
-  // if they started late: they go first,
-  // longest first.  When all of K and V fit in half of L2 the rest are
-  // ordered tile-major (later tiles first, the larger ones under a causal
-  // mask); otherwise K/V-group-major -- all tiles of the query heads that
-  // share one K/V head run together, so that head's K and V stay in L2 while
-  // they are reused -- longest first inside a group.  The query heads of a
-  // group are adjacent either way.
+  // if they started late.
   const int64_t heavy = std::max<int64_t>(1, total / (2 * std::max(ctas, 1)) / 2);
+  const int64_t share = total / std::max(ctas, 1);   // one CTA's share of the work
+
+  // Split tiles.  A tile whose list is far longer than the others (the rows
+  // of global tokens see every key) is cut into pieces of consecutive blocks,
+  // each a work unit of its own that writes an unnormalised partial result
+  // (O, row maximum, row sum) to a workspace slot; the CTA that finishes a
+  // tile's last piece combines them.  The pieces run beside the other units
+  // of their head, while that head's K and V are in L2, and spread the tile
+  // over many CTAs.  Automatic (max_unit_blocks = 0): pieces of
+  // P = max(32, 2 x median list) blocks for tiles longer than one CTA's share
+  // of the whole work (unsplit, such a tile alone would set the launch time)
+  // and than 2 P, within a 256 MiB workspace; max_unit_blocks > 0 cuts every
+  // list longer than that; < 0 never splits.
+  int64_t piece_len = 0;
+  if (max_unit_blocks > 0) {
+    piece_len = max_unit_blocks;
+  } else if (max_unit_blocks == 0 && n > 0) {
+    std::vector<int32_t> sorted(costs);
+    std::nth_element(sorted.begin(), sorted.begin() + sorted.size() / 2, sorted.end());
+    piece_len = std::max<int64_t>(32, 2 * int64_t(sorted[sorted.size() / 2]));
+  }
+  // piece: index into out->pieces, or -1; cost: the list length the order
+  // uses (for the pieces of a tile, the longest piece's, so that they stay
+  // together in list order)
+  struct Item { int32_t id, k0, n, piece, cost; };
+  std::vector<Item> items;
+  items.reserve(size_t(n));
+  out->pieces.clear();
+  out->split.clear();
+  int64_t slots = 0;
+  for (int64_t u = 0; u < n; ++u) {
+    const int32_t c = costs[size_t(u)];
+    bool split = false;
+    if (max_unit_blocks > 0) split = c > piece_len;
+    else if (max_unit_blocks == 0) split = c > share && c > 2 * piece_len;
+    const int64_t np = split ? (c + piece_len - 1) / piece_len : 1;
+    if (split && max_unit_blocks == 0 && (slots + np) * slot_bytes > (int64_t(256) << 20))
+      split = false;
+    if (!split) {
+      items.push_back({int32_t(u), 0, c, -1, c});
+      continue;
+    }
+    // np pieces of near-equal length
+    SplitTile st;
+    st.id = int32_t(u);
+    st.first_slot = int32_t(slots);
+    st.n_pieces = int32_t(np);
+    st.pad = 0;
+    out->split.push_back(st);
+    for (int64_t j = 0; j < np; ++j) {
+      const int32_t k0 = int32_t(j * c / np), k1 = int32_t((j + 1) * c / np);
+      Piece pc;
+      pc.id = int32_t(u);
+      pc.k0 = k0;
+      pc.n = k1 - k0;
+      pc.slot = int32_t(slots + j);
+      pc.split = int32_t(out->split.size() - 1);
+      pc.first_slot = int32_t(slots);
+      pc.n_pieces = int32_t(np);
+      pc.pad = 0;
+      items.push_back({int32_t(u), k0, k1 - k0, int32_t(out->pieces.size()),
+                       int32_t((c + np - 1) / np)});
+      out->pieces.push_back(pc);
+    }
+    slots += np;
+  }
+  out->n_slots = slots;
+
+  // Order: heavy units first, longest first.  When all of K and V fit in half
+  // of L2 the rest are ordered tile-major (later tiles first, the larger ones
+  // under a causal mask); otherwise K/V-group-major -- all tiles of the query
+  // heads that share one K/V head run together, so that head's K and V stay in
+  // L2 while they are reused -- longest first inside a group.  The query heads
+  // of a group are adjacent either way; the pieces of a split tile run in
+  // descending key order, like the tiles of their head.
   const bool group_major = kv_bytes > (int64_t(64) << 20);
   const int group = std::max(H / H_kv, 1);
-  std::stable_sort(units.begin(), units.end(), [&](int32_t a, int32_t b) {
-    const int ca = cost(a), cb = cost(b);
+  const int groups = std::max(H / group, 1);
+  // Group-major position of an item: its (b, K/V group) in queue order; the
+  // pieces of a split tile move one group earlier, so that they (and the merge
+  // their last one triggers) finish while their own group's tiles still run --
+  // also for the last group -- with their head's K and V read shortly before.
+  auto slot_of = [&](const Item& x) {
+    const int bh = x.id / T;
+    const int lg = (bh / H) * groups + (bh % H) / group;
+    return x.piece >= 0 ? std::max(lg - 1, 0) : lg;
+  };
+  std::stable_sort(items.begin(), items.end(), [&](const Item& x, const Item& y) {
+    const int ca = x.cost, cb = y.cost;
     const bool ha_ = ca > heavy, hb_ = cb > heavy;
     if (ha_ != hb_) return ha_;
     if (ha_ && ca != cb) return ca > cb;
-    const int bha = a / T, bhb = b / T;
+    const int bha = x.id / T, bhb = y.id / T;
     const int ba = bha / H, bb = bhb / H, ha = bha % H, hb = bhb % H;
     if (!ha_ && group_major) {
-      if (ba != bb) return ba < bb;
-      if (ha / group != hb / group) return ha / group < hb / group;
+      const int ga = slot_of(x), gb = slot_of(y);
+      if (ga != gb) return ga < gb;
       if (ca != cb) return ca > cb;
+      if (ha / group != hb / group) return ha / group < hb / group;
     }
-    const int ta = a % T, tb = b % T;
+    const int ta = x.id % T, tb = y.id % T;
     if (ta != tb) return ta > tb;
     if (ba != bb) return ba < bb;
-    return ha < hb;
+    if (ha != hb) return ha < hb;
+    return x.k0 > y.k0;
   });
+  out->units.resize(items.size());
+  for (size_t k = 0; k < items.size(); ++k)
+    out->units[k] = items[k].piece < 0 ? items[k].id : ~items[k].piece;
 }
 
 }  // namespace sa

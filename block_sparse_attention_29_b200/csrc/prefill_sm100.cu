@@ -95,6 +95,8 @@ struct Cfg {
 
 struct Unit {
   int b, r, h, hkv, t, beg, n;   // r: residue class of a dilated window (0 otherwise)
+  int slot;                      // piece of a split tile: its workspace slot; -1 otherwise
+  int split, first_slot, n_pieces;   // piece: its split tile and that tile's slots
 };
 
 struct Bars {
@@ -113,13 +115,27 @@ struct Bars {
   float red[3][4];     // per S buffer: warp maxima for the tile maximum
   Unit unit_slot[4];   // decoded work unit; n = -1 once the queue is exhausted
   uint32_t dec_val[4]; // decision ring: 1 = keep, 0 = skip
+  int merge_last;      // the piece just finished was its split tile's last
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block too large");
 
 
+template <bool SPLIT>
 __device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
   Unit u;
-  const int id = __ldg(p.units + ui);
+  int id = __ldg(p.units + ui), k0 = 0, n = -1;
+  u.slot = u.split = u.first_slot = u.n_pieces = -1;
+  if (SPLIT && id < 0) {   // a piece of a split tile
+    const int4 pc = __ldg(p.pieces + 2 * ~id);
+    const int4 st = __ldg(p.pieces + 2 * ~id + 1);
+    id = pc.x;
+    k0 = pc.y;
+    n = pc.z;
+    u.slot = pc.w;
+    u.split = st.x;
+    u.first_slot = st.y;
+    u.n_pieces = st.z;
+  }
   u.t = id % p.T;
   const int bh = id / p.T;
   u.h = bh % p.H;
@@ -128,8 +144,8 @@ __device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
   u.r = bd - u.b * p.dil;
   u.hkv = u.h / (p.H / p.Hkv);
   const int row = (p.head_pat ? u.h : 0) * p.T + u.t;
-  u.beg = __ldg(p.row_ptr + row);
-  u.n = __ldg(p.row_ptr + row + 1) - u.beg;
+  u.beg = __ldg(p.row_ptr + row) + k0;
+  u.n = n >= 0 ? n : __ldg(p.row_ptr + row + 1) - u.beg;
   return u;
 }
 
@@ -139,6 +155,7 @@ __device__ __forceinline__ Unit get_unit(const PrefillParams& p, int ui) {
 // softmax warps take the decoded units from the ring in the same order (so
 // they need no dependent global loads at unit boundaries).  n = -1 marks the
 // end of the queue.
+template <bool SPLIT>
 __device__ __forceinline__ bool publish_unit(const PrefillParams& p, Bars* bars, uint32_t n,
                                              Unit* out) {
   const uint32_t slot = n % kUnitRing;
@@ -148,13 +165,15 @@ __device__ __forceinline__ bool publish_unit(const PrefillParams& p, Bars* bars,
   const int v = atomicAdd(p.sched, 1);
   Unit u;
   if (v < p.n_units) {
-    u = get_unit(p, v);
+    u = get_unit<SPLIT>(p, v);
   } else {
     u.b = u.r = u.h = u.hkv = u.t = u.beg = 0;
     u.n = -1;
+    u.slot = u.split = u.first_slot = u.n_pieces = -1;
   }
   volatile int* d = reinterpret_cast<volatile int*>(&bars->unit_slot[slot]);
   d[0] = u.b; d[1] = u.h; d[2] = u.hkv; d[3] = u.t; d[4] = u.beg; d[5] = u.n; d[6] = u.r;
+  if (SPLIT) { d[7] = u.slot; d[8] = u.split; d[9] = u.first_slot; d[10] = u.n_pieces; }
   mbar_arrive(smem_u32(&bars->u_full[slot]));
   *out = u;
   return true;
@@ -163,6 +182,7 @@ __device__ __forceinline__ bool publish_unit(const PrefillParams& p, Bars* bars,
 // Consumer side: one thread (MMA, V loader) or every lane of a softmax warp
 // calls it; the slot is released once per caller group (the warp's lane 0
 // after the whole warp has read it).
+template <bool SPLIT>
 __device__ __forceinline__ bool take_unit(const PrefillParams& p, Bars* bars, uint32_t n, Unit* out,
                                           int where, bool whole_warp) {
   const uint32_t slot = n % kUnitRing;
@@ -172,6 +192,14 @@ __device__ __forceinline__ bool take_unit(const PrefillParams& p, Bars* bars, ui
   const volatile int* d = reinterpret_cast<const volatile int*>(&bars->unit_slot[slot]);
   out->b = d[0]; out->h = d[1]; out->hkv = d[2]; out->t = d[3]; out->beg = d[4]; out->n = d[5];
   out->r = d[6];
+  if (SPLIT) {
+    out->slot = d[7];
+    out->split = d[8];
+    out->first_slot = d[9];
+    out->n_pieces = d[10];
+  } else {
+    out->slot = out->split = out->first_slot = out->n_pieces = -1;
+  }
   if (whole_warp) {
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(&bars->u_empty[slot]));
@@ -182,7 +210,7 @@ __device__ __forceinline__ bool take_unit(const PrefillParams& p, Bars* bars, ui
 }
 
 // ------------------------------------------------------------ producer --
-template <int D>
+template <int D, bool SPLIT>
 __device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars) {
   using C = Cfg<D>;
   volatile int* abort_flag = &bars->abort;
@@ -191,7 +219,7 @@ __device__ void producer_role(const PrefillParams& p, uint8_t* smem, Bars* bars)
   uint32_t qc = 0, kc = 0;
   for (uint32_t n = 0;; ++n) {
     Unit u;
-    if (!publish_unit(p, bars, n, &u)) goto drain;
+    if (!publish_unit<SPLIT>(p, bars, n, &u)) goto drain;
     if (u.n < 0) break;
     if (u.n == 0) continue;
     if (!wait_bounded(smem_u32(&bars->q_empty), (qc & 1) ^ 1, abort_flag, p.err, W_PROD_Q))
@@ -229,7 +257,7 @@ drain:
 // Producer warp, lane 1: loads the V tile of every kept block, in block order,
 // as soon as a V stage is free.  With the rule on it takes each block's gate
 // decision from the decision ring first (skipped blocks load nothing).
-template <int D>
+template <int D, bool SPLIT>
 __device__ void vloader_role(const PrefillParams& p, uint8_t* smem, Bars* bars) {
   using C = Cfg<D>;
   volatile int* abort_flag = &bars->abort;
@@ -237,7 +265,7 @@ __device__ void vloader_role(const PrefillParams& p, uint8_t* smem, Bars* bars) 
   uint32_t vc = 0, g = 0;
   for (uint32_t n = 0;; ++n) {
     Unit u;
-    if (!take_unit(p, bars, n, &u, W_VL_UNIT, false)) goto drain;
+    if (!take_unit<SPLIT>(p, bars, n, &u, W_VL_UNIT, false)) goto drain;
     if (u.n < 0) break;
     for (int k = 0; k < u.n; ++k, ++g) {
       bool keep = true;
@@ -281,7 +309,7 @@ drain:
 //        in issue order);
 //   P  : take block k's P hand-off (kept or skipped) from the softmax;
 //   PV : O += P_k V_k for a kept block once V_k has landed.
-template <int D>
+template <int D, bool SPLIT>
 __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint32_t tmem) {
   using C = Cfg<D>;
   volatile int* abort_flag = &bars->abort;
@@ -296,7 +324,7 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
 
   for (uint32_t n = 0; ok; ++n) {
     Unit u;
-    if (!take_unit(p, bars, n, &u, W_MMA_UNIT, false)) {
+    if (!take_unit<SPLIT>(p, bars, n, &u, W_MMA_UNIT, false)) {
       ok = false;
       break;
     }
@@ -401,7 +429,109 @@ __device__ void mma_role(const PrefillParams& p, uint8_t* smem, Bars* bars, uint
   }
 }
 
+// Merge of a split tile's pieces for one row: the pieces' partial results
+// (O in the piece's scale m_j, row sum l_j; read past L1, they were written by
+// other CTAs) are brought to the largest m_j and summed; O / L -> bf16 and the
+// log-sum-exp as in the epilogue.  Pieces whose row saw no key (l_j = 0) are
+// left out.
 template <int D>
+__device__ __forceinline__ void merge_pieces(const PrefillParams& p, int first_slot, int n_pieces, int row,
+                             uint16_t* orow_ptr, float* lse_ptr) {
+  if (!orow_ptr) return;
+  const int64_t stride = int64_t(D + 2) * kTileQ;
+  const float* base = p.part + int64_t(first_slot) * stride + row;
+  // Loads are unconditional (a piece's O is finite, zero where its row saw no
+  // key) so that those of several pieces are in flight together.
+  float M = -INFINITY, L = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < n_pieces; ++j) {
+    const float* pj = base + j * stride;
+    const float mj = __ldcg(pj + D * kTileQ), lj = __ldcg(pj + (D + 1) * kTileQ);
+    if (lj > 0.f) {   // online merge of (M, L) with (m_j, l_j)
+      const float mn = fmaxf(M, mj);
+      L = L * ex2(M - mn) + lj * ex2(mj - mn);
+      M = mn;
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float acc[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) acc[q] = 0.f;
+#pragma unroll 2
+    for (int j = 0; j < n_pieces; ++j) {
+      const float* pj = base + j * stride;
+      const float mj = __ldcg(pj + D * kTileQ), lj = __ldcg(pj + (D + 1) * kTileQ);
+      float o[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q) o[q] = __ldcg(pj + (c0 + q) * kTileQ);
+      const float w = lj > 0.f ? ex2(mj - M) : 0.f;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) acc[q] = fmaf(w, o[q], acc[q]);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c0);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint4 o;
+      o.x = pack_bf16x2(acc[8 * v + 0] * inv, acc[8 * v + 1] * inv);
+      o.y = pack_bf16x2(acc[8 * v + 2] * inv, acc[8 * v + 3] * inv);
+      o.z = pack_bf16x2(acc[8 * v + 4] * inv, acc[8 * v + 5] * inv);
+      o.w = pack_bf16x2(acc[8 * v + 6] * inv, acc[8 * v + 7] * inv);
+      dst[v] = o;
+    }
+  }
+  if (lse_ptr) *lse_ptr = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+// Epilogue of a piece of a split tile (all four softmax warps): O
+// unnormalised (fp32), the row's scale reference m and its sum l go to the
+// piece's workspace slot, each column as 128 consecutive floats (one per row);
+// a piece with no kept block leaves O = 0.  The CTA that finishes the tile's
+// last piece (counted on a device-wide counter after a fence) merges them.
+// Kept out of line: it runs once per piece, and inlined it would take
+// registers from the block loop.  Returns false on a timed-out wait.
+template <int D>
+__device__ __noinline__ bool piece_epilogue(const PrefillParams& p, Bars* bars, uint32_t tmem_row,
+                                            const Unit& u, uint32_t kept, uint32_t pv_total,
+                                            float m, float l, int row, bool leader,
+                                            uint16_t* orow_ptr, float* lse_ptr) {
+  using C = Cfg<D>;
+  float* part = p.part + int64_t(u.slot) * (D + 2) * kTileQ + row;
+  if (kept > 0) {
+    const uint32_t last = pv_total - 1;
+    if (!wait_bounded(smem_u32(&bars->o_done[last % kODone]), (last / kODone) & 1, &bars->abort,
+                      p.err, W_SM_EPI))
+      return false;
+    tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tmem_row + C::TMEM_O + c * 32, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 32; ++q) __stcg(part + (c * 32 + q) * kTileQ, __uint_as_float(o[q]));
+    }
+    tc_fence_before();
+  } else {
+    for (int c = 0; c < D; ++c) __stcg(part + c * kTileQ, 0.f);
+  }
+  __stcg(part + D * kTileQ, m);
+  __stcg(part + (D + 1) * kTileQ, l);
+  __threadfence();
+  named_bar_sync(kSoftmaxBar, 128);
+  if (leader)
+    reinterpret_cast<volatile int*>(&bars->merge_last)[0] =
+        atomicAdd(p.split_cnt + u.split, 1) == u.n_pieces - 1;
+  named_bar_sync(kSoftmaxBar, 128);
+  if (reinterpret_cast<volatile int*>(&bars->merge_last)[0]) {
+    __threadfence();
+    merge_pieces<D>(p, u.first_slot, u.n_pieces, row, orow_ptr, lse_ptr);
+  }
+  return true;
+}
+
+template <int D, bool SPLIT>
 __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, int warp,
                              int lane) {
   using C = Cfg<D>;
@@ -415,7 +545,7 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
 
   for (uint32_t n = 0;; ++n) {
     Unit u;
-    if (!take_unit(p, bars, n, &u, W_SM_UNIT, true)) return;
+    if (!take_unit<SPLIT>(p, bars, n, &u, W_SM_UNIT, true)) return;
     if (u.n < 0) break;
     const int i = u.t * kTileQ + row;
     const bool row_ok = i < p.N;
@@ -587,6 +717,13 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
     }
 
     if (p.stats_only) continue;
+    if (SPLIT && u.slot >= 0) {
+      if (!piece_epilogue<D>(p, bars, tmem + lane_base, u, kept, pv_total, m, l, row, leader,
+                             row_ok ? p.O + orow * D : nullptr,
+                             row_ok && p.lse ? p.lse + orow : nullptr))
+        return;
+      continue;
+    }
     // Epilogue: O / l -> bf16, one row per thread.
     uint16_t* orow_ptr = p.O + orow * D;
     if (kept > 0) {
@@ -624,7 +761,7 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
   }
 }
 
-template <int D>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_constant__ PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -674,12 +811,12 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) producer_role<D>(p, smem, bars);
-    else if (lane == 1) vloader_role<D>(p, smem, bars);
+    if (lane == 0) producer_role<D, SPLIT>(p, smem, bars);
+    else if (lane == 1) vloader_role<D, SPLIT>(p, smem, bars);
   } else if (warp == 1) {
-    if (lane == 0) mma_role<D>(p, smem, bars, tmem);
+    if (lane == 0) mma_role<D, SPLIT>(p, smem, bars, tmem);
   } else {
-    softmax_role<D>(p, bars, tmem, warp, lane);
+    softmax_role<D, SPLIT>(p, bars, tmem, warp, lane);
   }
 
   tc_fence_before();
@@ -693,12 +830,14 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
     if (atomicAdd(p.sched + 1, 1) == int(gridDim.x) - 1) {
       atomicExch(p.sched, 0);
       atomicExch(p.sched + 1, 0);
+      if (SPLIT)
+        for (int k = 0; k < p.n_split; ++k) atomicExch(p.split_cnt + k, 0);
     }
   }
 }
 
 int g_num_sms[64] = {0};
-bool g_attr_set[2][64] = {{false}};
+bool g_attr_set[2][2][64] = {};
 
 }  // namespace
 
@@ -713,25 +852,20 @@ int launch_prefill(const PrefillParams& p, int d, cudaStream_t stream) {
   }
   if (p.n_units == 0) return SA_OK;
   const int grid = p.n_units < 2 * g_num_sms[dev] ? p.n_units : 2 * g_num_sms[dev];
-  if (d == 128) {
-    if (!g_attr_set[1][dev]) {
-      e = cudaFuncSetAttribute(prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg<128>::SMEM);
-      if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute");
-      g_attr_set[1][dev] = true;
-    }
-    prefill_kernel<128><<<grid, kThreads, Cfg<128>::SMEM, stream>>>(p);
-  } else if (d == 64) {
-    if (!g_attr_set[0][dev]) {
-      e = cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg<64>::SMEM);
-      if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute");
-      g_attr_set[0][dev] = true;
-    }
-    prefill_kernel<64><<<grid, kThreads, Cfg<64>::SMEM, stream>>>(p);
-  } else {
+  if (d != 128 && d != 64)
     return set_error(SA_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
+  // Plans without split tiles run the instantiation that has no piece code.
+  const bool split = p.n_split > 0;
+  bool& attr = g_attr_set[d == 128][split][dev];
+  const int smem = d == 128 ? Cfg<128>::SMEM : Cfg<64>::SMEM;
+  auto* kern = d == 128 ? (split ? prefill_kernel<128, true> : prefill_kernel<128, false>)
+                        : (split ? prefill_kernel<64, true> : prefill_kernel<64, false>);
+  if (!attr) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_error(e, "cudaFuncSetAttribute");
+    attr = true;
   }
+  kern<<<grid, kThreads, smem, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_error(e, "prefill launch");
   return SA_OK;

@@ -31,6 +31,11 @@ Workloads (names used by tests and bench):
                       and kept: the baseline of the rule's savings)
   bsfa_row_level      bsfa_causal's inputs and thresholds with the row-level reading of
                       the rule (rows also drop kept blocks below the threshold)
+  longformer_split    longformer_bigbird's inputs with the global rows' tiles cut into
+                      pieces of at most 34 blocks (plan option max_unit_blocks = 34)
+  bigbird_two_heads   longformer_bigbird's pattern on B=1 H=H_kv=2: the global rows'
+                      tile of each head is longer than a CTA's share of the launch
+                      (the automatic split cuts it)
 """
 from __future__ import annotations
 
@@ -62,6 +67,7 @@ class PrefillWorkload:
     dilation: int = 1
     skipped_in_denominator: int = 0   # block-skip variant (product pattern field)
     row_level_skip: int = 0           # block-skip rule, per-query reading (product pattern field)
+    max_unit_blocks: int = 0          # plan option: split tiles (0 automatic)
     # "calibrated": per-head thresholds from the calibration draw; "minus_inf":
     # thresholds of -inf (the rule computes and keeps every block: the run the
     # rule's savings are measured against)
@@ -145,6 +151,13 @@ WORKLOADS = {
                                       row_level_skip=1, seed=3000),
     "dilated_swa": PrefillWorkload("dilated_swa", B=1, H=32, H_kv=8, N=32768, d=128, causal=1,
                                    window=2048, dilation=8, block_q=128, block_k=64, seed=7000),
+    "longformer_split": PrefillWorkload("longformer_split", B=2, H=16, H_kv=16, N=65536, d=64,
+                                        causal=0, window=512, n_global=64, random_block=64,
+                                        n_random=3, block_q=128, block_k=64, max_unit_blocks=34,
+                                        seed=4000),
+    "bigbird_two_heads": PrefillWorkload("bigbird_two_heads", B=1, H=2, H_kv=2, N=65536, d=64,
+                                         causal=0, window=512, n_global=64, random_block=64,
+                                         n_random=3, block_q=128, block_k=64, seed=4000),
 }
 
 

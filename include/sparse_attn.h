@@ -143,6 +143,10 @@ typedef struct {
     int64_t blocks_desc;    /* listed blocks at the descriptor's block_q x block_k      */
     int64_t pairs;          /* sum over (b, h, i) of |G_i| of the static pattern        */
     double compile_ms;      /* host time spent compiling the pattern                    */
+    int64_t split_tiles;    /* tiles whose block list is cut into pieces (see
+                               sa_plan_options_t.max_unit_blocks)                       */
+    int64_t queue_units;    /* entries of the work queue: whole tiles plus pieces       */
+    int64_t workspace_bytes;/* device workspace of the pieces' partial results          */
 } sa_plan_info_t;
 
 /* Kernel choice for sparse_attn_plan_create_ex. */
@@ -166,6 +170,36 @@ int sparse_attn_plan_create(const sa_pattern_t *pat, int B, int H, int H_kv, int
  * other values: SA_ERR_INVALID_ARG). */
 int sparse_attn_plan_create_ex(const sa_pattern_t *pat, int B, int H, int H_kv, int N, int d,
                                int kernel, sa_plan_t **out);
+
+/* Plan options (sparse_attn_plan_create_opts).
+ *
+ * Split tiles: a query tile whose block list is far longer than the others
+ * (the rows of global tokens attend to every key) would run on one CTA while
+ * the other tiles of its head have long finished, and would read that head's
+ * K and V from HBM a second time.  Such a list is cut into pieces of
+ * consecutive blocks; each piece is a work unit of its own, scheduled beside
+ * the tiles of its head, that writes an unnormalised partial result (O in fp32,
+ * the row maximum and the row sum) to a device workspace owned by the plan; a
+ * merge kernel launched after the prefill combines the pieces of a tile (the
+ * same online-softmax combination the kernel applies across blocks) and writes
+ * O and the log-sum-exp.  Statistics, decisions and block masks are per block
+ * and do not depend on the split. */
+typedef struct {
+    int32_t kernel;           /* SA_KERNEL_*                                             */
+    int32_t max_unit_blocks;  /* 0: automatic -- a tile whose list is longer than one
+                                 CTA's share of the whole launch (it alone would set
+                                 the launch time) and than 2P blocks is cut into
+                                 pieces of about P = max(32, 2 x the median list
+                                 length) blocks, within a 256 MiB workspace; > 0:
+                                 every list longer than this many blocks is cut into
+                                 pieces of at most this many; < 0: no tile is split   */
+} sa_plan_options_t;
+
+/* Same as sparse_attn_plan_create with options (NULL: kernel SA_KERNEL_AUTO,
+ * max_unit_blocks 0).  Errors as sparse_attn_plan_create; SA_ERR_INVALID_ARG
+ * for an unknown kernel value. */
+int sparse_attn_plan_create_opts(const sa_pattern_t *pat, int B, int H, int H_kv, int N, int d,
+                                 const sa_plan_options_t *opts, sa_plan_t **out);
 int sparse_attn_plan_info(const sa_plan_t *plan, sa_plan_info_t *info);
 void sparse_attn_plan_destroy(sa_plan_t *plan);   /* synchronises the device; NULL ok */
 
@@ -312,6 +346,20 @@ int64_t sparse_attn_window_slot(int64_t j, int window, int n_global);
 int sparse_attn_prefill_noalloc(const void *Q, const void *K, const void *V, void *O,
                                 int B, int H, int H_kv, int N, int d, const sa_pattern_t *pat,
                                 float *lse_out, sa_stream_t stream);
+
+/* Host-only work order (no GPU needed): the prefill queue a plan built with
+ * these arguments and options->max_unit_blocks holds.  First call with
+ * units == NULL to get *n_units_out (queue entries), *n_pieces_out and
+ * *n_split_out; then again with units int32 [n_units], pieces int32
+ * [n_pieces][4] and split int32 [n_split][4].  units[k] >= 0 is a whole tile
+ * ((b'*H + h)*T + t, b' = b*k + residue with dilation k); units[k] < 0 is
+ * piece ~units[k] = {tile, first block of the list, blocks, workspace slot};
+ * split[s] = {tile, first slot, pieces, 0}.  Errors as sparse_attn_plan_create
+ * (no SA_ERR_CUDA / SA_ERR_NO_MEMORY). */
+int sparse_attn_work_order(const sa_pattern_t *pat, int B, int H, int H_kv, int N, int d,
+                           int max_unit_blocks, int64_t *n_units_out, int64_t *n_pieces_out,
+                           int64_t *n_split_out, int32_t *units, int32_t *pieces,
+                           int32_t *split);
 
 /* Host-only pattern compiler (no GPU needed): the block lists a plan holds, at
  * tile_q x tile_k granularity.  H_pat = H when random blocks are on, else 1
