@@ -19,6 +19,7 @@
 
 #include "common.h"
 #include "ptx.cuh"
+#include "softmax_util.cuh"
 
 namespace sa {
 namespace {
@@ -140,9 +141,17 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
     for (int u = 0; u < kUnroll; ++u) {
       float kf[8];
       bf16x8_to_f32(kv[u], kf);
-      float d = 0.f;
+      // the products in group_rows_update's order (even and odd dimensions
+      // in two chains, then their sum), as scalar instructions: the same
+      // roundings as its packed f32x2 form, so shared and per-head sets give
+      // the same bits; packed here measured slower
+      float d0 = q[0] * kf[0], d1 = q[1] * kf[1];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) d = fmaf(q[c], kf[c], d);
+      for (int c = 2; c < 8; c += 2) {
+        d0 = fmaf(q[c], kf[c], d0);
+        d1 = fmaf(q[c + 1], kf[c + 1], d1);
+      }
+      float d = d0 + d1;
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
       sc[u] = valid[u] ? d : -INFINITY;
@@ -206,7 +215,9 @@ __device__ __forceinline__ void group_rows_update(const float (&q)[G][8], float 
                                                   const uint4 (&vv)[kUnroll],
                                                   const bool (&valid)[kUnroll]) {
   constexpr int LPR = D / 8;
-  // Scores: each K row unpacked once, dotted with the G queries.
+  // Scores: each K row unpacked once, dotted with the G queries.  The
+  // products and the V accumulation run in packed f32x2 arithmetic (two
+  // lanes of a pair: even and odd dimensions).
   float sc[G][kUnroll];
 #pragma unroll
   for (int u = 0; u < kUnroll; ++u) {
@@ -214,9 +225,13 @@ __device__ __forceinline__ void group_rows_update(const float (&q)[G][8], float 
     bf16x8_to_f32(kv[u], kf);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float d = 0.f;
+      uint64_t d2 = f2_mul(f2_pack(q[g][0], q[g][1]), f2_pack(kf[0], kf[1]));
 #pragma unroll
-      for (int c = 0; c < 8; ++c) d = fmaf(q[g][c], kf[c], d);
+      for (int c = 2; c < 8; c += 2)
+        d2 = f2_fma(f2_pack(q[g][c], q[g][c + 1]), f2_pack(kf[c], kf[c + 1]), d2);
+      float d0, d1;
+      f2_unpack(d2, d0, d1);
+      float d = d0 + d1;
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
       sc[g][u] = valid[u] ? d : -INFINITY;
@@ -234,8 +249,12 @@ __device__ __forceinline__ void group_rows_update(const float (&q)[G][8], float 
     if (!live[g]) continue;
     const float alpha = ex2(m[g] - m_new);
     l[g] *= alpha;
+    const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[g][c] *= alpha;
+    for (int c = 0; c < 8; c += 2) {
+      const uint64_t r = f2_mul(f2_pack(acc[g][c], acc[g][c + 1]), a2);
+      f2_unpack(r, acc[g][c], acc[g][c + 1]);
+    }
     m[g] = m_new;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -251,8 +270,13 @@ __device__ __forceinline__ void group_rows_update(const float (&q)[G][8], float 
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       if (!live[g]) continue;
+      const uint64_t s2 = f2_pack(sc[g][u], sc[g][u]);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[g][c] = fmaf(sc[g][u], vf[c], acc[g][c]);
+      for (int c = 0; c < 8; c += 2) {
+        const uint64_t r =
+            f2_fma(s2, f2_pack(vf[c], vf[c + 1]), f2_pack(acc[g][c], acc[g][c + 1]));
+        f2_unpack(r, acc[g][c], acc[g][c + 1]);
+      }
     }
   }
 }

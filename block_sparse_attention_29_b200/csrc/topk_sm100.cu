@@ -28,6 +28,7 @@
 
 #include "common.h"
 #include "ptx.cuh"
+#include "softmax_util.cuh"
 
 namespace sa {
 namespace {
@@ -144,10 +145,14 @@ __global__ void __launch_bounds__(kScoreThreads, 2) topk_score_kernel(const Topk
       bf16x8_to_f32(kv[u], kf);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float d = 0.f;
+        // packed f32x2 products: even and odd dimensions, summed at the end
+        uint64_t d2 = f2_mul(f2_pack(q[g][0], q[g][1]), f2_pack(kf[0], kf[1]));
 #pragma unroll
-        for (int c = 0; c < 8; ++c) d = fmaf(q[g][c], kf[c], d);
-        v[u * G + g] = d;
+        for (int c = 2; c < 8; c += 2)
+          d2 = f2_fma(f2_pack(q[g][c], q[g][c + 1]), f2_pack(kf[c], kf[c + 1]), d2);
+        float d0, d1;
+        f2_unpack(d2, d0, d1);
+        v[u * G + g] = d0 + d1;
       }
     }
     // transposing reduction over the LPR lanes of each row
