@@ -253,9 +253,12 @@ struct SelectSmem {
   int32_t cand_j[kCandCap];
   uint32_t ws[33];
   int res[2];
-  uint32_t n_cand;
   uint32_t seg_sure[kSegs], seg_sel[kSegs], seg_tie[kSegs], seg_off[kSegs], tie_before[kSegs];
+  uint32_t seg_cand[kSegs];   // kept keys per segment (each in its warp's region)
+  int overflow;               // a segment held more kept keys than its region
 };
+// kept keys of a warp's segment: region [warp * kRegion, (warp + 1) * kRegion)
+constexpr int kRegion = kCandCap / kSegs;
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x) {
   const int lane = threadIdx.x & 31;
@@ -419,51 +422,74 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seg = (((len + kSegs - 1) / kSegs) + 127) & ~127;   // a multiple of 128 keys
   const int lo = warp * seg, hi = min(len, lo + seg);
-  if (threadIdx.x == 0) sm.n_cand = 0;
-  if (threadIdx.x < kSegs) sm.seg_sel[threadIdx.x] = sm.seg_tie[threadIdx.x] = 0;
+  if (threadIdx.x == 0) sm.overflow = 0;
   __syncthreads();
 
-  // sweep 1
-  uint32_t sure = 0;
-  for (int c0 = lo + lane * 4; c0 < hi; c0 += 128 * kSelUnroll) {
+  // sweep 1: keys above the bin counted per segment; the bin's keys (and
+  // indices) kept in the warp's own region of shared memory, placed by a warp
+  // prefix sum -- no shared counter, so no contended atomics
+  uint32_t sure = 0, wc = 0;   // wc: this warp's kept keys so far (warp-uniform)
+  uint32_t* ck = sm.cand_key + warp * kRegion;
+  int32_t* cj = sm.cand_j + warp * kRegion;
+  for (int c0 = lo; c0 < hi; c0 += 128 * kSelUnroll) {
     float4 v[kSelUnroll];
 #pragma unroll
     for (int u = 0; u < kSelUnroll; ++u) {
-      const int j0 = c0 + u * 128;
+      const int j0 = c0 + u * 128 + lane * 4;
       v[u] = j0 < hi ? *reinterpret_cast<const float4*>(sc + j0) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < kSelUnroll; ++u) {
-      const int j0 = c0 + u * 128;
+      if (c0 + u * 128 >= hi) break;   // the same for the whole warp
+      const int j0 = c0 + u * 128 + lane * 4;
       const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      bool cand[4] = {false, false, false, false};
+      uint32_t cl = 0;
       // most scores lie below the bin: one test per float4 skips them
-      if (!(fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])) >= f_lo)) continue;
+      if (fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])) >= f_lo) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (j0 + i < hi) {
-          if (x[i] >= f_hi) {
-            ++sure;
-          } else if (x[i] >= f_lo) {
-            const uint32_t slot = atomicAdd(&sm.n_cand, 1u);
-            if (slot < uint32_t(kCandCap)) {
-              sm.cand_key[slot] = topk_key(x[i]);
-              sm.cand_j[slot] = j0 + i;
-            }
-          }
+        for (int i = 0; i < 4; ++i) {
+          const bool in = j0 + i < hi;
+          const bool above = in && x[i] >= f_hi;
+          sure += above;
+          cand[i] = in && !above && x[i] >= f_lo;
+          cl += cand[i];
         }
       }
+      if (!__any_sync(0xffffffffu, cl != 0)) continue;
+      const uint32_t incl = warp_incl_scan(cl);
+      uint32_t pos = wc + incl - cl;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (cand[i]) {
+          if (pos < uint32_t(kRegion)) {
+            ck[pos] = topk_key(x[i]);
+            cj[pos] = j0 + i;
+          }
+          ++pos;
+        }
+      }
+      wc += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sure += __shfl_xor_sync(0xffffffffu, sure, o);
-  if (lane == 0) sm.seg_sure[warp] = sure;
+  if (lane == 0) {
+    sm.seg_sure[warp] = sure;
+    sm.seg_cand[warp] = wc;
+    if (wc > uint32_t(kRegion)) sm.overflow = 1;
+  }
   for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads) sm.h[i] = 0;
   __syncthreads();
-  const uint32_t nc = min(sm.n_cand, uint32_t(kCandCap));   // == c1
+  // a segment's kept keys overflowed its region: the generic path (its own sweeps)
+  if (sm.overflow) return select_generic(p, sm, sc, len, k, b1, r1, out, sh);
+  uint32_t nc = 0;
+  for (int w = 0; w < kSegs; ++w) nc += sm.seg_cand[w];   // == c1
 
   // level 2 and level 3 over the kept keys
-  for (uint32_t c = threadIdx.x; c < nc; c += kSelectThreads)
-    atomicAdd(&sm.h[(sm.cand_key[c] >> 10) & 2047u], 1u);
+  for (int c = threadIdx.x; c < kCandCap; c += kSelectThreads)
+    if (uint32_t(c % kRegion) < sm.seg_cand[c / kRegion])
+      atomicAdd(&sm.h[(sm.cand_key[c] >> 10) & 2047u], 1u);
   __syncthreads();
   find_bin<kTopkBins1>(sm.h, r1, sm.ws, sm.res);
   const int b2 = sm.res[0];
@@ -472,7 +498,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   const uint32_t pre = (uint32_t(b1) << 11) | uint32_t(b2 < 0 ? 0 : b2);
   for (int i = threadIdx.x; i < 1024; i += kSelectThreads) sm.h[i] = 0;
   __syncthreads();
-  for (uint32_t c = threadIdx.x; c < nc; c += kSelectThreads) {
+  for (int c = threadIdx.x; c < kCandCap; c += kSelectThreads) {
+    if (uint32_t(c % kRegion) >= sm.seg_cand[c / kRegion]) continue;
     const uint32_t key = sm.cand_key[c];
     if ((key >> 10) == pre) atomicAdd(&sm.h[key & 1023u], 1u);
   }
@@ -485,12 +512,24 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   const uint32_t thr = (pre << 10) | uint32_t(b3);
   const float f_thr = topk_key_float(thr);   // a score of the row, so a number
 
-  // kept keys above the threshold and keys equal to it, per segment
-  for (uint32_t c = threadIdx.x; c < nc; c += kSelectThreads) {
-    const uint32_t key = sm.cand_key[c];
-    const int sg = sm.cand_j[c] / seg;
-    if (key > thr) atomicAdd(&sm.seg_sel[sg], 1u);
-    else if (key == thr) atomicAdd(&sm.seg_tie[sg], 1u);
+  // kept keys above the threshold and keys equal to it, per segment: each
+  // warp counts its own region
+  {
+    uint32_t gt = 0, eq = 0;
+    for (uint32_t i = lane; i < wc; i += 32) {
+      const uint32_t key = ck[i];
+      gt += key > thr;
+      eq += key == thr;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      gt += __shfl_xor_sync(0xffffffffu, gt, o);
+      eq += __shfl_xor_sync(0xffffffffu, eq, o);
+    }
+    if (lane == 0) {
+      sm.seg_sel[warp] = gt;
+      sm.seg_tie[warp] = eq;
+    }
   }
   __syncthreads();
   if (warp == 0) {

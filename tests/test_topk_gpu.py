@@ -166,13 +166,16 @@ def test_topk_decode_full_size_sampled(product, oracle_mod, cuda):
 
 
 @pytest.mark.parametrize("L,top_k,two_levels", [(4096, 300, False), (20000, 100, False),
-                                                 (20000, 12000, True)],
-                         ids=["ties-over-segments", "overfull-bin", "overfull-bin-two-levels"])
+                                                 (20000, 12000, True), (32768, 500, "cluster")],
+                         ids=["ties-over-segments", "overfull-bin", "overfull-bin-two-levels",
+                              "clustered-bin"])
 def test_topk_decode_ties_in_index_order(product, oracle_mod, cuda, L, top_k, two_levels):
     """Equal scores are taken in index order when they span several of the
-    select pass's row segments, and when the threshold's first-level bin holds
-    more keys than shared memory keeps (its three-sweep path).  Checked exactly:
-    the near-cut tolerance of the other tests would accept any choice of ties."""
+    select pass's row segments, when the threshold's first-level bin holds
+    more keys than shared memory keeps (its three-sweep path), and when the
+    bin's keys crowd one segment beyond its share of shared memory (1000 equal
+    keys in the first of 32 segments).  Checked exactly: the near-cut
+    tolerance of the other tests would accept any choice of ties."""
     S, H, Hkv, d = 1, 2, 1, 128
     Q = _rand((S, H, d), L + top_k, cuda)
     Q[0, 1] = Q[0, 0]
@@ -180,7 +183,12 @@ def test_topk_decode_ties_in_index_order(product, oracle_mod, cuda, L, top_k, tw
     V = _rand((S, Hkv, L, d), L + top_k + 2, cuda)
     row_b = K[0, 0, 5].clone()
     K[0, 0] = row_b
-    if two_levels:
+    if two_levels == "cluster":
+        # keys 0..999 score higher (the same row plus the query direction)
+        row_a = (row_b.float() + Q[0, 0].float() / Q[0, 0].float().norm()).to(torch.bfloat16)
+        K[0, 0, :1000] = row_a
+        want = np.arange(top_k)
+    elif two_levels:
         # even keys score higher (the same row plus the query direction)
         row_a = (row_b.float() + Q[0, 0].float() / Q[0, 0].float().norm()).to(torch.bfloat16)
         K[0, 0, 0::2] = row_a
