@@ -59,7 +59,7 @@ typedef struct CUstream_st *sa_stream_t;
 enum {
     SA_OK = 0,
     SA_ERR_INVALID_ARG = 1,   /* bad pointer, shape, alignment or descriptor           */
-    SA_ERR_UNSUPPORTED = 2,   /* valid request this build has no kernel for            */
+    SA_ERR_UNSUPPORTED = 2,   /* valid request the library has no kernel for          */
     SA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed                      */
     SA_ERR_NO_MEMORY = 4,     /* host or device allocation failed                      */
     SA_ERR_TIMEOUT = 5,       /* device: a pipeline wait ran out of time; kernel bailed */
