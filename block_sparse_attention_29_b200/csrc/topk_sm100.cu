@@ -253,7 +253,7 @@ struct SelectSmem {
   int32_t cand_j[kCandCap];
   uint32_t ws[33];
   int res[2];
-  uint32_t seg_sure[kSegs], seg_sel[kSegs], seg_tie[kSegs], seg_off[kSegs], tie_before[kSegs];
+  uint32_t seg_sel[kSegs], seg_tie[kSegs], seg_off[kSegs], tie_before[kSegs];
   uint32_t seg_cand[kSegs];   // kept keys per segment (each in its warp's region)
   int overflow;               // a segment held more kept keys than its region
 };
@@ -417,7 +417,6 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   if (c1 > uint32_t(kCandCap) || b1 < 4 || b1 > 2043 || n_special != 0)
     return select_generic(p, sm, sc, len, k, b1, r1, out, sh);
   const float f_lo = topk_key_float(uint32_t(b1) << 21);        // x >= f_lo: bin >= b1
-  const float f_hi = topk_key_float(uint32_t(b1 + 1) << 21);    // x >= f_hi: bin >  b1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seg = (((len + kSegs - 1) / kSegs) + 127) & ~127;   // a multiple of 128 keys
@@ -425,10 +424,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   if (threadIdx.x == 0) sm.overflow = 0;
   __syncthreads();
 
-  // sweep 1: keys above the bin counted per segment; the bin's keys (and
-  // indices) kept in the warp's own region of shared memory, placed by a warp
-  // prefix sum -- no shared counter, so no contended atomics
-  uint32_t sure = 0, wc = 0;   // wc: this warp's kept keys so far (warp-uniform)
+  // The one sweep: every key at or above the threshold's bin (the keys above
+  // it are all selected, the bin's are resolved below) is kept with its index
+  // in the warp's own region of shared memory, in index order, placed by a
+  // warp prefix sum -- no shared counter, so no contended atomics.
+  uint32_t wc = 0;   // this warp's kept keys so far (warp-uniform)
   uint32_t* ck = sm.cand_key + warp * kRegion;
   int32_t* cj = sm.cand_j + warp * kRegion;
   for (int c0 = lo; c0 < hi; c0 += 128 * kSelUnroll) {
@@ -443,17 +443,14 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
       if (c0 + u * 128 >= hi) break;   // the same for the whole warp
       const int j0 = c0 + u * 128 + lane * 4;
       const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      bool cand[4] = {false, false, false, false};
+      bool keep[4] = {false, false, false, false};
       uint32_t cl = 0;
       // most scores lie below the bin: one test per float4 skips them
       if (fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])) >= f_lo) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const bool in = j0 + i < hi;
-          const bool above = in && x[i] >= f_hi;
-          sure += above;
-          cand[i] = in && !above && x[i] >= f_lo;
-          cl += cand[i];
+          keep[i] = j0 + i < hi && x[i] >= f_lo;
+          cl += keep[i];
         }
       }
       if (!__any_sync(0xffffffffu, cl != 0)) continue;
@@ -461,7 +458,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
       uint32_t pos = wc + incl - cl;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (cand[i]) {
+        if (keep[i]) {
           if (pos < uint32_t(kRegion)) {
             ck[pos] = topk_key(x[i]);
             cj[pos] = j0 + i;
@@ -472,10 +469,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
       wc += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sure += __shfl_xor_sync(0xffffffffu, sure, o);
   if (lane == 0) {
-    sm.seg_sure[warp] = sure;
     sm.seg_cand[warp] = wc;
     if (wc > uint32_t(kRegion)) sm.overflow = 1;
   }
@@ -483,13 +477,13 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   __syncthreads();
   // a segment's kept keys overflowed its region: the generic path (its own sweeps)
   if (sm.overflow) return select_generic(p, sm, sc, len, k, b1, r1, out, sh);
-  uint32_t nc = 0;
-  for (int w = 0; w < kSegs; ++w) nc += sm.seg_cand[w];   // == c1
 
-  // level 2 and level 3 over the kept keys
-  for (int c = threadIdx.x; c < kCandCap; c += kSelectThreads)
-    if (uint32_t(c % kRegion) < sm.seg_cand[c / kRegion])
-      atomicAdd(&sm.h[(sm.cand_key[c] >> 10) & 2047u], 1u);
+  // level 2 and level 3 over the bin's keys
+  for (int c = threadIdx.x; c < kCandCap; c += kSelectThreads) {
+    if (uint32_t(c % kRegion) >= sm.seg_cand[c / kRegion]) continue;
+    const uint32_t key = sm.cand_key[c];
+    if ((key >> 21) == uint32_t(b1)) atomicAdd(&sm.h[(key >> 10) & 2047u], 1u);
+  }
   __syncthreads();
   find_bin<kTopkBins1>(sm.h, r1, sm.ws, sm.res);
   const int b2 = sm.res[0];
@@ -508,27 +502,29 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   const int b3 = sm.res[0];
   const uint32_t take_eq = uint32_t(sm.res[1]);   // keys equal to the threshold to take
   __syncthreads();
-  if (b2 < 0 || b3 < 0 || nc != c1) return select_failed(p, sh, 5);
+  if (b2 < 0 || b3 < 0) return select_failed(p, sh, 5);
   const uint32_t thr = (pre << 10) | uint32_t(b3);
-  const float f_thr = topk_key_float(thr);   // a score of the row, so a number
 
-  // kept keys above the threshold and keys equal to it, per segment: each
-  // warp counts its own region
+  // per segment: its kept keys above the threshold and equal to it, and the
+  // bin's keys (whose total must be the bin's count)
   {
-    uint32_t gt = 0, eq = 0;
+    uint32_t gt = 0, eq = 0, in_bin = 0;
     for (uint32_t i = lane; i < wc; i += 32) {
       const uint32_t key = ck[i];
       gt += key > thr;
       eq += key == thr;
+      in_bin += (key >> 21) == uint32_t(b1);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       gt += __shfl_xor_sync(0xffffffffu, gt, o);
       eq += __shfl_xor_sync(0xffffffffu, eq, o);
+      in_bin += __shfl_xor_sync(0xffffffffu, in_bin, o);
     }
     if (lane == 0) {
-      sm.seg_sel[warp] = gt;
+      sm.seg_sel[warp] = gt;   // above the threshold: the keys above the bin included
       sm.seg_tie[warp] = eq;
+      sm.seg_cand[warp] = in_bin;
     }
   }
   __syncthreads();
@@ -537,61 +533,36 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
     const uint32_t tie = sm.seg_tie[lane];
     const uint32_t tie_before = warp_incl_scan(tie) - tie;
     const uint32_t taken = take_eq > tie_before ? min(tie, take_eq - tie_before) : 0u;
-    const uint32_t tot = sm.seg_sure[lane] + sm.seg_sel[lane] + taken;
+    const uint32_t tot = sm.seg_sel[lane] + taken;
     const uint32_t incl = warp_incl_scan(tot);
     sm.seg_off[lane] = incl - tot;
     sm.tie_before[lane] = tie_before;
-    if (lane == 31) sm.res[0] = int(incl);
+    const uint32_t nb = warp_incl_scan(sm.seg_cand[lane]);
+    if (lane == 31) {
+      sm.res[0] = int(incl);
+      sm.res[1] = int(nb);
+    }
   }
   __syncthreads();
+  if (uint32_t(sm.res[1]) != c1) return select_failed(p, sh, 5);   // the bin's count
 
-  // sweep 2: the selected indices of each segment, in order
+  // the output: each warp walks its kept keys in index order and writes the
+  // selected ones' indices at its segment's offset
   uint32_t run = sm.seg_off[warp];
   uint32_t tie_run = sm.tie_before[warp];
-  for (int c0 = lo; c0 < hi; c0 += 128 * kSelUnroll) {
-    float4 v[kSelUnroll];
-#pragma unroll
-    for (int u = 0; u < kSelUnroll; ++u) {
-      const int j0 = c0 + u * 128 + lane * 4;
-      v[u] = j0 < hi ? *reinterpret_cast<const float4*>(sc + j0) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kSelUnroll; ++u) {
-      if (c0 + u * 128 >= hi) break;   // the same for the whole warp
-      const int j0 = c0 + u * 128 + lane * 4;
-      const float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      bool gt[4] = {false, false, false, false}, eq[4] = {false, false, false, false};
-      uint32_t ct = 0;
-      if (fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3])) >= f_thr) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const bool in = j0 + i < hi;
-          gt[i] = in && x[i] > f_thr;
-          eq[i] = in && x[i] == f_thr;
-          ct += eq[i];
-        }
-      }
-      uint32_t tr = tie_run;
-      if (__any_sync(0xffffffffu, ct != 0)) {
-        const uint32_t incl = warp_incl_scan(ct);
-        tr += incl - ct;
-        tie_run += __shfl_sync(0xffffffffu, incl, 31);
-      }
-      bool sel[4];
-      uint32_t cs = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        sel[i] = gt[i] || (eq[i] && tr < take_eq);
-        tr += eq[i];
-        cs += sel[i];
-      }
-      const uint32_t incl = warp_incl_scan(cs);
-      uint32_t pos = run + incl - cs;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (sel[i] && pos < uint32_t(k)) out[pos++] = j0 + i;
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (uint32_t c = 0; c < wc; c += 32) {
+    const uint32_t i = c + lane;
+    const uint32_t key = i < wc ? ck[i] : 0u;
+    const bool gt = i < wc && key > thr;
+    const bool eq = i < wc && key == thr;
+    const uint32_t eq_b = __ballot_sync(0xffffffffu, eq);
+    const bool sel = gt || (eq && tie_run + __popc(eq_b & lt) < take_eq);
+    const uint32_t sel_b = __ballot_sync(0xffffffffu, sel);
+    const uint32_t pos = run + __popc(sel_b & lt);
+    if (sel && pos < uint32_t(k)) out[pos] = cj[i];
+    run += __popc(sel_b);
+    tie_run += __popc(eq_b);
   }
   if (threadIdx.x == 0) {
     const uint32_t total = uint32_t(sm.res[0]);
