@@ -118,12 +118,17 @@ def _sample_rows(B, H, N, n_random, seed):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["mistral_swa", "longformer_bigbird", "dilated_swa"])
+@pytest.mark.parametrize("name", ["mistral_swa", "longformer_bigbird", "dilated_swa",
+                                  "longformer_split", "bigbird_two_heads"])
 def test_prefill_full_size_sampled(product, oracle_mod, cuda, name):
+    """The benchmark's launch of each workload (split tiles included: the
+    sampled rows 0, 1 and 127 are global rows, whose tile is split)."""
     w = WORKLOADS[name]
     Q, K, V, tab = prefill_inputs(w, device=cuda)
     plan = product.Plan(product.Pattern(**w.pattern_fields(), random_table=tab), w.B, w.H, w.H_kv,
-                        w.N, w.d)
+                        w.N, w.d, max_unit_blocks=w.max_unit_blocks)
+    if name in ("longformer_split", "bigbird_two_heads"):
+        assert plan.info["split_tiles"] == w.B * w.H
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=cuda)
     O = plan.prefill(Q, K, V, lse=lse)
     product.check_device_error()
