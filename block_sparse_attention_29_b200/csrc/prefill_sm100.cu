@@ -54,7 +54,10 @@ constexpr uint32_t kUnitRing = 4;       // depth of the work-unit ring
 // consumers of a ring slot: the MMA thread, the V loader and one lane of
 // each softmax warp
 constexpr uint32_t kUnitConsumers = 1 + 1 + 4;
-constexpr uint32_t kDecRing = 4;        // depth of the gate-decision ring
+// The block-skip gate: each softmax warp publishes its warp maximum of a
+// block in a ring of kRedRing slots (an mbarrier per slot counts the four
+// warps); the V loader reads the four and decides, and frees the slot.
+constexpr uint32_t kRedRing = 8;
 // PV completions are tracked on a ring of kODone barriers (PV number n on
 // barrier n % kODone, phase n / kODone).  A softmax warp waits on PV number L
 // only after the S of its current block has landed, and S(k) is issued after
@@ -105,16 +108,15 @@ struct Bars {
   uint64_t v_full[3], v_empty[3];
   uint64_t s_full[3];                   // per S buffer: S of the block written
   uint64_t p_ready[3];                  // per S buffer: P written (or block skipped)
-  uint64_t dec_full[4], dec_empty[4];   // gate decisions, softmax -> V loader
+  uint64_t red_full[kRedRing], red_empty[kRedRing];   // warp maxima: softmax -> V loader
   uint64_t o_done[4];
   uint64_t drain;
   uint64_t u_full[4], u_empty[4];   // work-unit ring (producer -> MMA + softmax)
   uint32_t tmem_base;
   int abort;
   uint32_t flags[3];   // per S buffer: 1 = block kept, 0 = skipped
-  float red[3][4];     // per S buffer: warp maxima for the tile maximum
+  float red[kRedRing][4];   // per ring slot: the four warp maxima of a block
   Unit unit_slot[4];   // decoded work unit; n = -1 once the queue is exhausted
-  uint32_t dec_val[4]; // decision ring: 1 = keep, 0 = skip
   int merge_last;      // the piece just finished was its split tile's last
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block too large");
@@ -255,8 +257,8 @@ drain:
 
 // ------------------------------------------------------------- V loader --
 // Producer warp, lane 1: loads the V tile of every kept block, in block order,
-// as soon as a V stage is free.  With the rule on it takes each block's gate
-// decision from the decision ring first (skipped blocks load nothing).
+// as soon as a V stage is free.  With the rule on it first takes the block's
+// decision from its four warp maxima (skipped blocks load nothing).
 template <int D, bool SPLIT>
 __device__ void vloader_role(const PrefillParams& p, uint8_t* smem, Bars* bars) {
   using C = Cfg<D>;
@@ -268,17 +270,21 @@ __device__ void vloader_role(const PrefillParams& p, uint8_t* smem, Bars* bars) 
     if (!take_unit<SPLIT>(p, bars, n, &u, W_VL_UNIT, false)) goto drain;
     if (u.n < 0) break;
     for (int k = 0; k < u.n; ++k, ++g) {
+      const int e = __ldg(p.entries + u.beg + k);
+      const int kb = e >> 1;
       bool keep = true;
       if (p.gate) {
-        const uint32_t slot = g % kDecRing;
-        if (!wait_bounded(smem_u32(&bars->dec_full[slot]), (g / kDecRing) & 1, abort_flag, p.err,
+        // the rule's decision, from the four warp maxima (as the softmax warps take it)
+        const uint32_t rs = g % kRedRing;
+        if (!wait_bounded(smem_u32(&bars->red_full[rs]), (g / kRedRing) & 1, abort_flag, p.err,
                           W_VL_DEC))
           goto drain;
-        keep = reinterpret_cast<volatile uint32_t*>(bars->dec_val)[slot] != 0;
-        mbar_arrive(smem_u32(&bars->dec_empty[slot]));
+        const volatile float* r = bars->red[rs];
+        const float tmax = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+        mbar_arrive(smem_u32(&bars->red_empty[rs]));
+        keep = !p.stats_only && ((e & 1) || !(tmax * p.scale < __ldg(p.thresholds + u.h)));
       }
       if (!keep) continue;
-      const int kb = __ldg(p.entries + u.beg + k) >> 1;
       const uint32_t vs = vc % C::VS;
       if (!wait_bounded(smem_u32(&bars->v_empty[vs]), ((vc / C::VS) & 1) ^ 1, abort_flag, p.err,
                         W_VL_EMPTY))
@@ -572,12 +578,13 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
       // neither reads S nor computes exponentials: its rows' P is zero.
       const bool none =
           C::kSkipInvisible && p.n_random > 0 && partial && __all_sync(0xffffffffu, vis == 0ull);
-      // The leader claims this block's decision-ring slot now, while S is
-      // still being computed (the V loader frees slots as it reads them).
-      bool slot_ok = true;
-      if (leader && p.gate)
-        slot_ok = wait_bounded(smem_u32(&bars->dec_empty[g % kDecRing]),
-                               ((g / kDecRing) & 1) ^ 1, abort_flag, p.err, W_SM_DEC);
+      // This block's slot of the maxima ring, claimed now while S is still
+      // being computed (the V loader frees slots as it reads them).
+      const uint32_t rs = g % kRedRing;
+      if (p.want_stats && p.gate &&
+          !wait_bounded(smem_u32(&bars->red_empty[rs]), ((g / kRedRing) & 1) ^ 1, abort_flag,
+                        p.err, W_SM_DEC))
+        return;
       // S of this block is in S buffer fb; the MMA thread computes the next
       // block's S into the other buffer meanwhile.
       const uint32_t tS = tmem + lane_base + kTmemS + 64 * fb;
@@ -602,34 +609,39 @@ __device__ void softmax_role(const PrefillParams& p, Bars* bars, uint32_t tmem, 
 
       bool keep = true;
       if (p.want_stats) {
+        // The tile maximum is the largest of the four warp maxima: each warp
+        // publishes its own; a warp whose own maximum keeps the block (a
+        // tile maximum is at least as large) needs nobody else's, the others
+        // wait for all four.  No barrier between the warps.
         const float wm = warp_max(mx);
-        if (lane == 0) bars->red[fb][q4] = wm;
-        // Past this barrier every warp has read its rows of S (a skipped
-        // block is handed off by the leader alone, after which the MMA thread
-        // may overwrite the buffer).
-        tc_fence_before();
-        named_bar_sync(kSoftmaxBar, 128);
-        const float tmax = fmaxf(fmaxf(bars->red[fb][0], bars->red[fb][1]),
-                                 fmaxf(bars->red[fb][2], bars->red[fb][3]));
+        if (lane == 0) reinterpret_cast<volatile float*>(bars->red[rs])[q4] = wm;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->red_full[rs]));
+        const bool own_keep = p.gate && !p.stats_only && (partial || !(wm * p.scale < tau));
+        const bool need_all = (warp == 2 && (p.stat_out || p.mask_out)) || (p.gate && !own_keep);
+        float tmax = wm;
+        if (need_all) {
+          if (!wait_bounded(smem_u32(&bars->red_full[rs]), (g / kRedRing) & 1, abort_flag, p.err,
+                            W_SM_P))
+            return;
+          const volatile float* r = bars->red[rs];
+          tmax = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+        }
         const float stat = tmax * p.scale;
         if (p.gate) keep = !p.stats_only && (partial || !(stat < tau));
         if (leader) {
           if (p.stat_out) p.stat_out[tile_base + kb] = stat;
           if (p.mask_out) p.mask_out[tile_base + kb] = keep || p.stats_only ? 1 : 2;
-          if (p.gate) {
-            flags[fb] = keep ? 1u : 0u;
-            if (slot_ok) {
-              const uint32_t slot = g % kDecRing;
-              reinterpret_cast<volatile uint32_t*>(bars->dec_val)[slot] = keep ? 1u : 0u;
-              mbar_arrive(smem_u32(&bars->dec_full[slot]));
-            }
-          }
         }
+        if (p.gate && lane == 0) flags[fb] = keep ? 1u : 0u;   // every warp: the same value
       } else if (leader && p.mask_out) {
         p.mask_out[tile_base + kb] = 1;
       }
       if (!keep) {
-        if (leader) mbar_arrive_cnt(smem_u32(&bars->p_ready[fb]), kSoftmaxWarps);
+        // each warp hands back its rows of the S buffer, already read
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[fb]));
         // Default rule: the block's keys leave G.  Variant: they stay in the
         // denominator -- the max and the row sum below take them, no P is
         // written (the S buffer is already handed back) and no PV runs.
@@ -784,9 +796,9 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
     }
     for (uint32_t b = 0; b < kODone; ++b) mbar_init(smem_u32(&bars->o_done[b]), 1);
     mbar_init(smem_u32(&bars->drain), 1);
-    for (uint32_t r = 0; r < kDecRing; ++r) {
-      mbar_init(smem_u32(&bars->dec_full[r]), 1);
-      mbar_init(smem_u32(&bars->dec_empty[r]), 1);
+    for (uint32_t r = 0; r < kRedRing; ++r) {
+      mbar_init(smem_u32(&bars->red_full[r]), kSoftmaxWarps);
+      mbar_init(smem_u32(&bars->red_empty[r]), 1);
     }
     for (uint32_t r = 0; r < kUnitRing; ++r) {
       mbar_init(smem_u32(&bars->u_full[r]), 1);
