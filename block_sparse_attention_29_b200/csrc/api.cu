@@ -637,10 +637,11 @@ int sparse_attn_decode_window(const void* Q, const void* K, const void* V,
 
 namespace {
 // Workspace of the top-k decode: scores [S*H][Lp] fp32, first-level
-// histograms [S*H][kTopkBins1], selected keys [S*H][top_k] and counts [S*H];
-// each region starts on a 256-byte boundary.
+// histograms [S*H][kTopkBins1], selected keys [S*H][top_k], counts [S*H] and
+// the selected keys' scores [S*H][top_k] fp32; each region starts on a
+// 256-byte boundary.
 struct TopkLayout {
-  size_t scores = 0, hist = 0, idx = 0, idx_len = 0, total = 0;
+  size_t scores = 0, hist = 0, idx = 0, idx_len = 0, sel = 0, total = 0;
 };
 size_t round_up256(size_t n) { return (n + 255) & ~size_t(255); }
 bool topk_layout(int S, int H, int L, int top_k, TopkLayout* t) {
@@ -651,7 +652,8 @@ bool topk_layout(int S, int H, int L, int top_k, TopkLayout* t) {
   t->hist = round_up256(sh * Lp * 4);
   t->idx = t->hist + round_up256(sh * kTopkBins1 * 4);
   t->idx_len = t->idx + round_up256(sh * size_t(top_k) * 4);
-  t->total = t->idx_len + round_up256(sh * 4);
+  t->sel = t->idx_len + round_up256(sh * 4);
+  t->total = t->sel + round_up256(sh * size_t(top_k) * 4);
   return true;
 }
 }  // namespace
@@ -699,6 +701,7 @@ int sparse_attn_decode_topk(const void* Q, const void* K, const void* V, const i
   p.hist = reinterpret_cast<uint32_t*>(w + t.hist);
   p.idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + t.idx);
   p.idx_len = idx_len_out ? idx_len_out : reinterpret_cast<int32_t*>(w + t.idx_len);
+  p.sel_scores = reinterpret_cast<float*>(w + t.sel);
   p.S = S;
   p.H = H;
   p.Hkv = H_kv;

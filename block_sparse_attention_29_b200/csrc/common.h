@@ -115,6 +115,7 @@ struct TopkParams {
   uint32_t* hist;            // workspace [S][H][kTopkBins1]
   int32_t* idx;              // [S][H][top_k] selected keys, ascending
   int32_t* idx_len;          // [S][H] selected count
+  float* sel_scores;         // workspace [S][H][top_k]: the selected keys' scores
   int S, H, Hkv, L, Lp, top_k, chunk;   // Lp: L rounded up to a multiple of 4
   float scale_log2;
   int* err;                  // device error word

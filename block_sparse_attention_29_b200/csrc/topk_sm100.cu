@@ -308,7 +308,7 @@ __device__ __forceinline__ void select_failed(const TopkParams& p, int sh, int s
 // block-wide prefix sums.
 __device__ __noinline__ void select_generic(const TopkParams& p, SelectSmem& sm, const float* sc,
                                             int len, int k, int b1, uint32_t r1, int32_t* out,
-                                            int sh) {
+                                            float* sel_out, int sh) {
   uint32_t* h = sm.h;
   for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads) h[i] = 0;
   __syncthreads();
@@ -365,7 +365,10 @@ __device__ __noinline__ void select_generic(const TopkParams& p, SelectSmem& sm,
     uint32_t pos = n_out + block_excl_scan(cs, sm.ws, &sel_total);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (sel[i] && pos < uint32_t(k)) out[pos++] = j0 + i;
+      if (sel[i] && pos < uint32_t(k)) {
+        out[pos] = j0 + i;
+        sel_out[pos++] = x[i];
+      }
     n_out += sel_total;
     n_eq += eq_total;
   }
@@ -389,8 +392,13 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   const int len = seq_len(p, s, 4);
   const int k = min(p.top_k, len);
   int32_t* out = p.idx + (int64_t)sh * p.top_k;
+  float* sel_out = p.sel_scores + (int64_t)sh * p.top_k;
   if (k == len) {   // every key is selected
-    for (int j = threadIdx.x; j < len; j += kSelectThreads) out[j] = j;
+    const float* scr = p.scores + (int64_t)sh * p.Lp;
+    for (int j = threadIdx.x; j < len; j += kSelectThreads) {
+      out[j] = j;
+      sel_out[j] = scr[j];
+    }
     if (threadIdx.x == 0) p.idx_len[sh] = len;
     return;
   }
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   // infinity or NaN (bins 0-3 and 2044-2047), which the key order ranks but
   // float comparisons do not.
   if (c1 > uint32_t(kCandCap) || b1 < 4 || b1 > 2043 || n_special != 0)
-    return select_generic(p, sm, sc, len, k, b1, r1, out, sh);
+    return select_generic(p, sm, sc, len, k, b1, r1, out, sel_out, sh);
   const float f_lo = topk_key_float(uint32_t(b1) << 21);        // x >= f_lo: bin >= b1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -476,7 +484,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
   for (int i = threadIdx.x; i < kTopkBins1; i += kSelectThreads) sm.h[i] = 0;
   __syncthreads();
   // a segment's kept keys overflowed its region: the generic path (its own sweeps)
-  if (sm.overflow) return select_generic(p, sm, sc, len, k, b1, r1, out, sh);
+  if (sm.overflow) return select_generic(p, sm, sc, len, k, b1, r1, out, sel_out, sh);
 
   // level 2 and level 3 over the bin's keys
   for (int c = threadIdx.x; c < kCandCap; c += kSelectThreads) {
@@ -560,7 +568,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
     const bool sel = gt || (eq && tie_run + __popc(eq_b & lt) < take_eq);
     const uint32_t sel_b = __ballot_sync(0xffffffffu, sel);
     const uint32_t pos = run + __popc(sel_b & lt);
-    if (sel && pos < uint32_t(k)) out[pos] = cj[i];
+    if (sel && pos < uint32_t(k)) {
+      out[pos] = cj[i];
+      sel_out[pos] = topk_key_float(key);   // the score itself (the key transform is a bijection)
+    }
     run += __popc(sel_b);
     tie_run += __popc(eq_b);
   }
@@ -573,9 +584,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) topk_select_kernel(const To
 
 // --------------------------------------------------------------- attend --
 // One CTA per (sequence, head): rows of the selected set split over row
-// groups of D/8 lanes; each group keeps an online softmax over the stored
-// scores (already log2-scaled) and accumulates its V rows; groups merge
-// through shared memory.
+// groups of D/8 lanes; each group keeps an online softmax over the selected
+// keys' scores (already log2-scaled, written contiguously by the select pass)
+// and accumulates its V rows; groups merge through shared memory.
 template <int D>
 __global__ void __launch_bounds__(kAttendThreads) topk_attend_kernel(const TopkParams p) {
   constexpr int LPR = D / 8;
@@ -588,7 +599,7 @@ __global__ void __launch_bounds__(kAttendThreads) topk_attend_kernel(const TopkP
   const int grp = threadIdx.x / LPR, gl = threadIdx.x % LPR;
   const int len = p.idx_len[sh];
   const int32_t* idx = p.idx + (int64_t)sh * p.top_k;
-  const float* sc = p.scores + (int64_t)sh * p.Lp;
+  const float* sel = p.sel_scores + (int64_t)sh * p.top_k;   // the selected keys' scores
   const uint16_t* Vb = p.V + ((int64_t)s * p.Hkv + hkv) * p.L * D + gl * 8;
 
   float m = -INFINITY, l = 0.f, acc[8];
@@ -603,7 +614,7 @@ __global__ void __launch_bounds__(kAttendThreads) topk_attend_kernel(const TopkP
       int j = r < len ? __ldg(idx + r) : -1;
       if (j >= p.L) j = -1;   // cannot happen: the select pass writes indices < len
       vv[u] = j >= 0 ? ld_stream(Vb + (int64_t)j * D) : make_uint4(0, 0, 0, 0);
-      w[u] = j >= 0 ? __ldg(sc + j) : -INFINITY;
+      w[u] = j >= 0 ? __ldg(sel + r) : -INFINITY;
     }
     float mx = w[0];
 #pragma unroll

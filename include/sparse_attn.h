@@ -310,8 +310,9 @@ int sparse_attn_decode_window(const void *Q, const void *K, const void *V,
  *            it is written; calls that overlap on the GPU need separate ones.
  *   scale: 0 means 1/sqrt(d).
  * Three kernels on `stream` (a score pass that reads every K row once per K/V
- * head, an exact radix select, an attention pass over the selected V rows)
- * plus a memset of the workspace histogram.  Errors: SA_ERR_INVALID_ARG
+ * head, an exact radix select that also writes the selected keys' scores, an
+ * attention pass over the selected V rows and those scores) plus a memset of
+ * the workspace histogram.  Errors: SA_ERR_INVALID_ARG
  * (shapes, H % H_kv, top_k < 1, alignment, workspace too small),
  * SA_ERR_UNSUPPORTED (d not 64/128, sizes past 32-bit grid limits). */
 size_t sparse_attn_decode_topk_workspace(int S, int H, int L, int top_k);

@@ -126,7 +126,8 @@ def test_decode_entry_points_reject_bad_arguments_on_host(product):
     def r256(n):
         return (n + 255) // 256 * 256
     Lp = (Lk + 3) // 4 * 4
-    want = r256(S * H * Lp * 4) + r256(S * H * 2048 * 4) + r256(S * H * k * 4) + r256(S * H * 4)
+    want = (r256(S * H * Lp * 4) + r256(S * H * 2048 * 4) + r256(S * H * k * 4) + r256(S * H * 4)
+            + r256(S * H * k * 4))
     assert product.decode_topk_workspace_bytes(S, H, Lk, k) == want
     assert product.decode_topk_workspace_bytes(S, H, Lk, 0) == 0
 
