@@ -12,15 +12,20 @@
 // One CTA = 6 warps, persistent, two CTAs per SM (each owns 256 TMEM columns):
 //   warp 0      TMA producer: lane 0 loads the Q tile once per work unit and
 //               the K blocks into a ring; lane 1 loads the V tiles of kept
-//               blocks (after the gate decision when the rule is on).
+//               blocks (when the rule is on, after deciding from the softmax
+//               warps' four maxima of the block).
 //   warp 1      TMEM owner and single-thread tcgen05 issuer: S = Q K^T into
 //               TMEM, O += P V with P read from TMEM, as an event loop that
 //               issues whichever step is ready.
 //   warps 2..5  softmax warpgroup, one query row per thread (TMEM lane):
-//               mask of partial blocks, row max, tile max and gate, online
-//               softmax statistics (m, l) in fp32, P (bf16) written to TMEM,
-//               lazy rescale of O, epilogue O / l.
-// Work units (b, h, tile) come from a launch-wide queue: the host orders them
+//               mask of partial blocks, row max, the warp's maximum published
+//               for the gate (a warp waits for the other three only when its
+//               own does not keep the block), online softmax statistics
+//               (m, l) in fp32, P (bf16) written to TMEM, lazy rescale of O,
+//               epilogue O / l.
+// Work units (b, h, tile) -- or pieces of a split tile's block list, whose
+// partial results the CTA finishing the last piece merges -- come from a
+// launch-wide queue: the host orders them
 // (very long units first; then tile-major when all of K/V fits in L2, else
 // K/V-group-major so a K/V head's blocks stay in L2 while its query heads use
 // them) and each CTA's producer claims the next one with an atomic counter
