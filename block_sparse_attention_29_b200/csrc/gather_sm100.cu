@@ -219,6 +219,8 @@ __device__ __forceinline__ void group_rows_update(const float (&q)[G][8], float 
   // products and the V accumulation run in packed f32x2 arithmetic (two
   // lanes of a pair: even and odd dimensions).
   float sc[G][kUnroll];
+  constexpr int NV = G * kUnroll;   // partial dots per lane: value u * G + g
+  float pv[NV];
 #pragma unroll
   for (int u = 0; u < kUnroll; ++u) {
     float kf[8];
@@ -231,10 +233,40 @@ __device__ __forceinline__ void group_rows_update(const float (&q)[G][8], float 
         d2 = f2_fma(f2_pack(q[g][c], q[g][c + 1]), f2_pack(kf[c], kf[c + 1]), d2);
       float d0, d1;
       f2_unpack(d2, d0, d1);
-      float d = d0 + d1;
+      pv[u * G + g] = d0 + d1;
+    }
+  }
+  if constexpr (NV >= LPR) {
+    // Transposing reduction over the row's LPR lanes: at each level a lane
+    // keeps half of its values and adds its partner's copy of them, so lane l
+    // ends with the totals of values l*HV .. l*HV + HV - 1 (NV - 1 shuffles
+    // instead of NV * log2(LPR)); every total is the same pairwise tree as a
+    // butterfly's, so the bits do not change.  Then each total is read from
+    // its lane.
+    constexpr int HV = NV / LPR;
+#pragma unroll
+    for (int o = LPR / 2, half = NV / 2; o > 0; o >>= 1, half >>= 1) {
+      const bool upper = (threadIdx.x & o) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float keep = upper ? pv[half + i] : pv[i];
+        const float send = upper ? pv[i] : pv[half + i];
+        pv[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    const int base = (threadIdx.x & 31) & ~(LPR - 1);   // the row group's first lane
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const float d = __shfl_sync(0xffffffffu, pv[v % HV], base + v / HV);
+      sc[v % G][v / G] = valid[v / G] ? d : -INFINITY;
+    }
+  } else {
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      float d = pv[v];
 #pragma unroll
       for (int o = LPR / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-      sc[g][u] = valid[u] ? d : -INFINITY;
+      sc[v % G][v / G] = valid[v / G] ? d : -INFINITY;
     }
   }
   // Online softmax per head; sc becomes the weights.
