@@ -343,6 +343,8 @@ int64_t sparse_attn_window_slot(int64_t j, int window, int n_global);
  * device address (with that device current); make it before any stream
  * capture.  Every call reuses the array: calls that can overlap on the GPU
  * (different streams without ordering) race; calls on one stream do not.
+ * No tile is split into pieces here (the pieces' workspace would not fit the
+ * array): every tile is one work unit, as with max_unit_blocks < 0.
  * Calls no cudaMalloc, cudaFree or other allocating library routine. */
 int sparse_attn_prefill_noalloc(const void *Q, const void *K, const void *V, void *O,
                                 int B, int H, int H_kv, int N, int d, const sa_pattern_t *pat,
