@@ -118,3 +118,47 @@ def test_automatic_split_leaves_even_workloads_alone(product):
                    (product.Pattern(causal=1), 32768)):
         units, pieces, split = product.work_order(pat, 1, 32, 8, N, 128, 0)
         assert len(split) == 0 and len(units) == 32 * (N // 128)
+
+
+def _lens(product, pat, H, N, units, T):
+    row_ptr, kb, full, cnt, H_pat, _ = product.compile_pattern(pat, H, N)
+    out = []
+    for u in units:
+        h, t = (u // T) % H, u % T
+        r = (h if H_pat > 1 else 0) * T + t
+        out.append(int(row_ptr[r + 1] - row_ptr[r]))
+    return np.array(out)
+
+
+def test_order_long_units_first_then_tile_major(product):
+    """K and V within half of L2 (tile-major): units longer than half a CTA's
+    share of the work come first, longest first; the rest by descending tile,
+    the query heads of a tile in order."""
+    B, H, Hkv, N, d = 1, 4, 2, 8192, 128   # K + V = 8 MiB
+    pat = product.Pattern(causal=1)
+    units, pieces, split = product.work_order(pat, B, H, Hkv, N, d, -1)
+    T = N // 128
+    lens = _lens(product, pat, H, N, units, T)
+    heavy = max(1, lens.sum() // (2 * 296) // 2)
+    n_heavy = int((lens > heavy).sum())
+    assert np.all(lens[:n_heavy] > heavy) and np.all(np.diff(lens[:n_heavy]) <= 0)
+    rest = units[n_heavy:]
+    t = rest % T
+    assert np.all(np.diff(t) <= 0)                         # descending tile
+    for tt in np.unique(t):
+        hs = (rest[t == tt] // T) % H
+        assert np.array_equal(hs, np.sort(hs))             # heads of a tile in order
+
+
+def test_order_kv_group_major_when_kv_exceeds_half_of_l2(product):
+    """K and V above half of L2: the tiles of one K/V group (its query heads)
+    run together, longest first inside the group."""
+    B, H, Hkv, N, d = 1, 8, 4, 65536, 128  # K + V = 128 MiB
+    pat = product.Pattern(causal=1, window=1024)
+    units, pieces, split = product.work_order(pat, B, H, Hkv, N, d, -1)
+    T = N // 128
+    group = (units // T) % H // (H // Hkv)
+    assert np.all(np.diff(group) >= 0)
+    lens = _lens(product, pat, H, N, units, T)
+    for g in np.unique(group):
+        assert np.all(np.diff(lens[group == g]) <= 0)
