@@ -253,7 +253,7 @@ def setup_prefill(w, device, torch, sa, workloads):
     return dict(step=step, e2e_step=lambda s: e2e_step(host, dev_bufs, s), h2d=h2d, d2h=d2h,
                 flops=computed, exact_flops=exact, dense_flops=dense, algo_bytes=algo_bytes,
                 extra=extra, kernel="prefill_kernel",
-                launches_per_step=2 if plan.info["split_tiles"] else 1,
+                launches_per_step=1,  # split tiles are merged inside the same launch
                 kernel_files=["prefill_sm100.cu", "softmax_util.cuh", "ptx.cuh", "common.h",
                               "pattern_compiler.cu"],
                 metric="effective TFLOP/s (computed blocks)", unit="TFLOP/s", bound="tensor",
