@@ -177,13 +177,15 @@ int sparse_attn_plan_create_ex(const sa_pattern_t *pat, int B, int H, int H_kv, 
  * (the rows of global tokens attend to every key) would run on one CTA while
  * the other tiles of its head have long finished, and would read that head's
  * K and V from HBM a second time.  Such a list is cut into pieces of
- * consecutive blocks; each piece is a work unit of its own, scheduled beside
- * the tiles of its head, that writes an unnormalised partial result (O in fp32,
- * the row maximum and the row sum) to a device workspace owned by the plan; a
- * merge kernel launched after the prefill combines the pieces of a tile (the
+ * consecutive blocks; each piece is a work unit of its own, queued with the
+ * tiles of the K/V group before its own, that writes an unnormalised partial
+ * result (O in fp32, the row maximum and the row sum) to a device workspace
+ * owned by the plan.  Inside the same launch, the CTA that finishes the last
+ * piece of a tile (a device-wide counter per tile) combines the pieces (the
  * same online-softmax combination the kernel applies across blocks) and writes
- * O and the log-sum-exp.  Statistics, decisions and block masks are per block
- * and do not depend on the split. */
+ * O and the log-sum-exp; the counters are back at zero when the launch ends.
+ * Statistics, decisions and block masks are per block and do not depend on the
+ * split. */
 typedef struct {
     int32_t kernel;           /* SA_KERNEL_*                                             */
     int32_t max_unit_blocks;  /* 0: automatic -- a tile whose list is longer than one
