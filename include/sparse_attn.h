@@ -230,7 +230,9 @@ int sparse_attn_prefill_plan(const sa_plan_t *plan, const void *Q, const void *K
 /* One-shot prefill: looks the pattern up in a per-process plan cache (keyed on
  * every descriptor field, the random table's contents and the shapes), compiles
  * it on a miss (synchronous, see sparse_attn_plan_create), then launches as
- * sparse_attn_prefill_plan with pat->thresholds. */
+ * sparse_attn_prefill_plan with pat->thresholds.  Calls that hit the same
+ * cached plan share its work-queue counters, so they must not overlap on the
+ * GPU either (one stream, or ordered streams). */
 int sparse_attn_prefill(const void *Q, const void *K, const void *V, void *O,
                         int B, int H, int H_kv, int N, int d, const sa_pattern_t *pat,
                         float *lse_out, uint8_t *block_mask_out, sa_stream_t stream);
