@@ -101,7 +101,17 @@ def _check_tensor(name, t, shape, dtype):
         raise ValueError(f"{name} must be contiguous")
     if t.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor")
-    del torch
+    # the library launches on the current device: a tensor of another device
+    # would hand its kernels a pointer into that device's memory
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on cuda:{t.device.index}, the current device is cuda:{cur}")
+
+
+def _tiles(N: int):
+    """(T_q, n_kb) of the block-mask and block-statistics layouts: 128-row query
+    tiles and 64-key blocks."""
+    return (N + 127) // 128, (N + 63) // 64
 
 
 KERNEL_AUTO = 0            # the kernel measured fastest for the shape (single-head today)
@@ -176,6 +186,9 @@ class Plan:
         if block_stat is None:
             block_stat = torch.full((self.B, self.H, self.T, self.n_kb), float("-inf"),
                                     dtype=torch.float32, device=Q.device)
+        _check_tensor("block_stat", block_stat, (self.B, self.H, self.T, self.n_kb), torch.float32)
+        if block_mask is not None:
+            _check_tensor("block_mask", block_mask, (self.B, self.H, self.T, self.n_kb), torch.uint8)
         check(lib().sparse_attn_block_stats(self._h, _ptr(Q), _ptr(K), _ptr(block_stat),
                                             _ptr(block_mask), _stream(stream)))
         return block_stat
@@ -183,8 +196,10 @@ class Plan:
     def calibrate(self, block_stat, q: float = 0.5, out=None, stream=None):
         """Per-head thresholds (rank floor((n-1) q) of full-block statistics)."""
         import torch
+        _check_tensor("block_stat", block_stat, (self.B, self.H, self.T, self.n_kb), torch.float32)
         if out is None:
             out = torch.empty(self.H, dtype=torch.float32, device=block_stat.device)
+        _check_tensor("out", out, (self.H,), torch.float32)
         check(lib().sparse_attn_calibrate(self._h, _ptr(block_stat), float(q), _ptr(out),
                                           _stream(stream)))
         return out
@@ -202,6 +217,12 @@ def sparse_attn_prefill(Q, K, V, pattern: Pattern, thresholds=None, O=None, lse=
     if O is None:
         O = torch.empty_like(Q)
     _check_tensor("O", O, (B, H, N, d), torch.bfloat16)
+    if thresholds is not None:
+        _check_tensor("thresholds", thresholds, (H,), torch.float32)
+    if lse is not None:
+        _check_tensor("lse", lse, (B, H, N), torch.float32)
+    if block_mask is not None:
+        _check_tensor("block_mask", block_mask, (B, H) + _tiles(N), torch.uint8)
     st, _tab = pattern.to_c(_ptr(thresholds) or 0)
     check(lib().sparse_attn_prefill(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), B, H, Hkv, N, d,
                                     ctypes.byref(st), _ptr(lse), _ptr(block_mask),
@@ -223,6 +244,8 @@ def sparse_attn_prefill_noalloc(Q, K, V, pattern: Pattern, O, thresholds=None, l
     _check_tensor("K", K, (B, Hkv, N, d), torch.bfloat16)
     _check_tensor("V", V, (B, Hkv, N, d), torch.bfloat16)
     _check_tensor("O", O, (B, H, N, d), torch.bfloat16)
+    if thresholds is not None:
+        _check_tensor("thresholds", thresholds, (H,), torch.float32)
     if lse is not None:
         _check_tensor("lse", lse, (B, H, N), torch.float32)
     st, _tab = pattern.to_c(_ptr(thresholds) or 0)
